@@ -1,0 +1,480 @@
+#!/usr/bin/env python3
+"""Throughput of the NF4 + double-quant QLoRA frozen-base linear layer on B200.
+
+One step = the hot path of one 65B-shape decoder layer (q/k/v/o 8192x8192,
+gate/up 22016x8192, down 8192x22016; NF4 blocks of 64 with FP8 double
+quantization; LoRA r = 64, alpha = 16) over 8192 tokens per GPU:
+
+  * forward + backward of q, k, v (shared input, dX accumulated) and o;
+  * the SiLU-gated MLP: gate and up forward, h = silu(g) * u, down forward,
+    then down backward, SiLU-gate backward, gate and up backward (dX accumulated);
+  * forward of all seven projections at M = 16 tokens (weight-stream bound);
+  * with N > 1 ranks (data parallel, 8192 tokens per rank): an all-reduce of
+    every adapter gradient dA, dB over NCCL.
+
+The weights are quantized once before timing (the pages quantize the frozen
+base once, offline); quantize / dequantize throughput is measured as separate
+components. Inputs are seeded synthetic tensors.
+
+Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & tokens/s (7B/65B shapes), % of roofline"
+WORKLOAD = "65B-shape decoder linears (q/k/v/o 8192x8192, gate/up 22016x8192, down 8192x22016), NF4+DQ, r=64"
+M_TOKENS = 8192
+M_SMALL = 16
+RANK_R = 64
+ALPHA = 16.0
+LAYERS = [("q_proj", 8192, 8192), ("k_proj", 8192, 8192), ("v_proj", 8192, 8192), ("o_proj", 8192, 8192),
+          ("gate_proj", 22016, 8192), ("up_proj", 22016, 8192), ("down_proj", 8192, 22016)]
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ------------------------------------------------------------------ helpers --
+def linear_flops(m: int, n: int, k: int, r: int, backward: bool) -> float:
+    """Algorithmic flops: forward 2MNK + 2Mr(K+N); backward adds dX (2MNK + 2MKr),
+    G = dY B (2MNr), dB (2MNr) and dA (2MKr). No dequant work, no dW."""
+    f = 2.0 * m * n * k + 2.0 * m * r * (k + n)
+    if backward:
+        f += 2.0 * m * n * k + 4.0 * m * r * (k + n)
+    return f
+
+
+def step_flops(m: int = M_TOKENS, m_small: int = M_SMALL, r: int = RANK_R) -> float:
+    total = 0.0
+    for _, n, k in LAYERS:
+        total += linear_flops(m, n, k, r, True) + linear_flops(m_small, n, k, r, False)
+    return total
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "_source": "fallback"}
+
+
+def max_over_ranks(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_reduce_grads(flat) -> None:
+    """Data-parallel exchange: sum the adapter gradients of every rank."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self) -> dict:
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax = float(parts[2].split()[0])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------- CPU oracle leg --
+class OracleSample:
+    """The oracle on a bounded sample of the workload: q_proj (8192 x 8192,
+    r = 64) with the weight quantized and dequantized once (setup), then per
+    step: forward for `rows` sampled tokens, backward dX for those rows, and
+    the adapter gradients dA, dB over all 8192 tokens."""
+
+    def __init__(self, rows: int = 32):
+        from bit_nf4_quantized_03_b200 import synth
+        from oracle import nf4_oracle as o
+        self.o = o
+        name, n, k = LAYERS[0]
+        W = synth.weight(n, k, layer=0)
+        self.Wd = o.dequantize_f64(o.quantize(W.numpy(), o.MODE_DQ_FP8), (n, k))
+        self.X = synth.activations(M_TOKENS, k, layer=0)
+        self.A, self.B = synth.lora_pair(RANK_R, k, n, layer=0)
+        self.dY = synth.grad_output(M_TOKENS, n, layer=0)
+        self.rows = synth.sample_rows(M_TOKENS, rows).numpy()
+        m = M_TOKENS
+        r = RANK_R
+        nr = len(self.rows)
+        self.flops = (2.0 * nr * n * k + 2.0 * nr * r * (k + n)        # Y rows
+                      + 2.0 * nr * n * k + 2.0 * nr * r * k            # dX rows
+                      + 2.0 * m * n * r + 2.0 * m * k * r              # G, U over all tokens
+                      + 2.0 * m * n * r + 2.0 * m * k * r)             # dB, dA
+        self.desc = (f"q_proj 8192x8192 r=64: forward and dX for {nr} sampled token rows of 8192, "
+                     f"dA/dB over all 8192 tokens (fp64 numpy); weight quantized/dequantized once before timing")
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        self.o.linear_forward(self.Wd, self.X, self.A, self.B, ALPHA, rows=self.rows)
+        self.o.linear_backward(self.Wd, self.X, self.dY, self.A, self.B, ALPHA, dx_rows=self.rows)
+        return time.perf_counter() - t0
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s = OracleSample()
+    for _ in range(args.warmup):
+        s.step()
+    times = [s.step() for _ in range(args.steps)]
+    total = sum(times)
+    value = s.flops * len(times) / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": s.desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": s.desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ native arm --
+class Workload:
+    def __init__(self, dev):
+        import torch
+        import bit_nf4_quantized_03_b200 as q
+        from bit_nf4_quantized_03_b200 import synth
+        self.q, self.dev = q, dev
+        rank = int(os.environ.get("RANK", "0"))
+        off = 1000 * rank                      # every rank gets its own tokens
+        bf, f32 = torch.bfloat16, torch.float32
+        self.w, self.A, self.B = {}, {}, {}
+        for i, (name, n, k) in enumerate(LAYERS):
+            W = synth.weight(n, k, layer=i).to(dev)
+            qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+            q.qlora_nf4_quantize(W, qw)
+            del W
+            a, b = synth.lora_pair(RANK_R, k, n, layer=i)
+            self.w[name], self.A[name], self.B[name] = qw, a.to(dev), b.to(dev)
+        torch.cuda.synchronize()
+        M, H, I = M_TOKENS, 8192, 22016
+        # host copies (pinned) of every input a step consumes
+        self.host = {
+            "x_attn": synth.activations(M, H, layer=off + 10), "x_o": synth.activations(M, H, layer=off + 11),
+            "x_mlp": synth.activations(M, H, layer=off + 12),
+            "dy_q": synth.grad_output(M, H, layer=off + 20), "dy_k": synth.grad_output(M, H, layer=off + 21),
+            "dy_v": synth.grad_output(M, H, layer=off + 22), "dy_o": synth.grad_output(M, H, layer=off + 23),
+            "dy_mlp": synth.grad_output(M, H, layer=off + 24),
+            "x16": synth.activations(M_SMALL, H, layer=off + 30), "h16": synth.activations(M_SMALL, I, layer=off + 31),
+        }
+        self.host = {k_: v.pin_memory() for k_, v in self.host.items()}
+        self.d = {k_: v.to(dev) for k_, v in self.host.items()}
+        e = lambda *s, dt=bf: torch.empty(*s, dtype=dt, device=dev)
+        self.y = {nm: e(M, n) for nm, n, _ in LAYERS if nm not in ("gate_proj", "up_proj", "down_proj")}
+        self.g, self.u, self.h, self.y_mlp = e(M, I), e(M, I), e(M, I), e(M, H)
+        self.dh, self.dg, self.du = e(M, I), e(M, I), e(M, I)
+        self.dx_attn, self.dx_o, self.dx_mlp = e(M, H), e(M, H), e(M, H)
+        self.U = {nm: e(M, RANK_R, dt=f32) for nm, _, _ in LAYERS}
+        self.y16 = {nm: e(M_SMALL, n) for nm, n, _ in LAYERS}
+        # adapter gradients live in one flat buffer (one all-reduce for the data-parallel exchange)
+        sizes = [RANK_R * k + n * RANK_R for _, n, k in LAYERS]
+        self.grads = torch.zeros(sum(sizes), dtype=f32, device=dev)
+        self.dA, self.dB, o_ = {}, {}, 0
+        for (nm, n, k), sz in zip(LAYERS, sizes):
+            self.dA[nm] = self.grads[o_:o_ + RANK_R * k].view(RANK_R, k)
+            self.dB[nm] = self.grads[o_ + RANK_R * k:o_ + sz].view(n, RANK_R)
+            o_ += sz
+        self.host_grads = torch.empty(self.grads.shape, dtype=f32).pin_memory()
+        ws = max(max(q.qlora_linear_workspace_bytes(M, n, k, RANK_R),
+                     q.qlora_linear_workspace_bytes(M_SMALL, n, k, RANK_R)) for _, n, k in LAYERS)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.host.values())
+        self.d2h_bytes = self.host_grads.numel() * 4
+
+    def _fwd(self, nm, X, Y, U):
+        q = self.q
+        q.qlora_linear_fwd(self.w[nm], X, self.A[nm], self.B[nm], RANK_R, ALPHA, Y, q.QLORA_DTYPE_BF16, U, self.ws)
+
+    def _bwd(self, nm, X, dY, dX, acc_dx):
+        q = self.q
+        flags = q.QLORA_BWD_ACCUMULATE_DX if acc_dx else 0
+        q.qlora_linear_bwd(self.w[nm], X, dY, self.A[nm], self.B[nm], RANK_R, ALPHA, self.U[nm], dX,
+                           q.QLORA_DTYPE_BF16, self.dA[nm], self.dB[nm], flags, self.ws)
+
+    def step(self):
+        q, d = self.q, self.d
+        for nm in ("q_proj", "k_proj", "v_proj"):
+            self._fwd(nm, d["x_attn"], self.y[nm], self.U[nm])
+        self._fwd("o_proj", d["x_o"], self.y["o_proj"], self.U["o_proj"])
+        self._fwd("gate_proj", d["x_mlp"], self.g, self.U["gate_proj"])
+        self._fwd("up_proj", d["x_mlp"], self.u, self.U["up_proj"])
+        q.qlora_silu_gate_fwd(self.g, self.u, self.h)
+        self._fwd("down_proj", self.h, self.y_mlp, self.U["down_proj"])
+        self._bwd("down_proj", self.h, d["dy_mlp"], self.dh, False)
+        q.qlora_silu_gate_bwd(self.dh, self.g, self.u, self.dg, self.du)
+        self._bwd("gate_proj", d["x_mlp"], self.dg, self.dx_mlp, False)
+        self._bwd("up_proj", d["x_mlp"], self.du, self.dx_mlp, True)
+        self._bwd("o_proj", d["x_o"], d["dy_o"], self.dx_o, False)
+        self._bwd("q_proj", d["x_attn"], d["dy_q"], self.dx_attn, False)
+        self._bwd("k_proj", d["x_attn"], d["dy_k"], self.dx_attn, True)
+        self._bwd("v_proj", d["x_attn"], d["dy_v"], self.dx_attn, True)
+        for nm, _, _ in LAYERS:
+            x = d["h16"] if nm == "down_proj" else d["x16"]
+            self._fwd(nm, x, self.y16[nm], None)
+        all_reduce_grads(self.grads)
+
+    def h2d(self):
+        for k_, v in self.host.items():
+            self.d[k_].copy_(v, non_blocking=True)
+
+    def d2h(self):
+        self.host_grads.copy_(self.grads, non_blocking=True)
+
+
+def time_steps(fn, steps, flush=None, sync_barrier=None):
+    """Device time of `steps` calls of fn (CUDA events on the current stream),
+    L2 flushed between calls outside the events. Returns ms per call."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if sync_barrier:
+        sync_barrier()
+    torch.cuda.synchronize()
+    for a, b in evs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    if sync_barrier:
+        sync_barrier()
+    return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+
+def components(dev, peaks) -> dict:
+    """Quantize / dequantize (4096 x 4096 with outliers) and M = 16 forward of
+    the 65B q_proj, each against the measured HBM copy bandwidth."""
+    import torch
+    import bit_nf4_quantized_03_b200 as q
+    from bit_nf4_quantized_03_b200 import synth
+    out = {}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    W = synth.weight(4096, 4096, outlier_frac=0.001).to(dev)
+    ne = W.numel()
+    for mode, tag in ((q.QLORA_SCALE_BF16, "bf16"), (q.QLORA_SCALE_DQ_FP8, "dq_fp8")):
+        qw = q.QuantizedWeight(4096, 4096, mode, device=dev)
+        ws = torch.empty(max(1, q.qlora_nf4_quantize_workspace_bytes(4096, 4096, mode)), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda: q.qlora_nf4_quantize(W, qw, ws)
+        for _ in range(3):
+            fn()
+        ms = time_steps(fn, 20, flush)
+        scale_b = 2.0 / 64 if mode == q.QLORA_SCALE_BF16 else 1.0 / 64 + 4.0 / 16384
+        algo = ne * (4.0 + 0.5 + scale_b)
+        out[f"quantize_{tag}"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
+                                  "algo_bytes": algo}
+        o_ = torch.empty(4096, 4096, dtype=torch.bfloat16, device=dev)
+        fn = lambda: q.qlora_nf4_dequantize(qw, o_)
+        for _ in range(3):
+            fn()
+        ms = time_steps(fn, 20, flush)
+        algo = ne * (0.5 + scale_b + 2.0)
+        out[f"dequantize_{tag}"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6,
+                                    "frac": algo / ms / 1e6 / peaks["hbm_gbs"], "algo_bytes": algo}
+    # weight-stream bound forward at M = 16 (65B q_proj)
+    n, k = 8192, 8192
+    W = synth.weight(n, k).to(dev)
+    qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+    q.qlora_nf4_quantize(W, qw)
+    del W
+    a, b = synth.lora_pair(RANK_R, k, n)
+    a, b = a.to(dev), b.to(dev)
+    x = synth.activations(M_SMALL, k).to(dev)
+    y = torch.empty(M_SMALL, n, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(q.qlora_linear_workspace_bytes(M_SMALL, n, k, RANK_R), dtype=torch.uint8, device=dev)
+    fn = lambda: q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, None, ws)
+    for _ in range(3):
+        fn()
+    ms = time_steps(fn, 50, flush)
+    algo = n * k * (0.5 + 1.0 / 64 + 4.0 / 16384) + 2.0 * M_SMALL * (k + n) + 2.0 * RANK_R * (k + n)
+    out["fwd_m16_q_proj"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
+                             "algo_bytes": algo}
+    return out
+
+
+def run_native(args) -> None:
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from bit_nf4_quantized_03_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import bit_nf4_quantized_03_b200 as q
+    peaks = measured_peaks()
+    barrier = (lambda: dist.barrier()) if world > 1 else None
+
+    wl = Workload(dev)
+    for _ in range(args.warmup):
+        wl.step()
+    q.qlora_check_device_error()
+
+    # timed region: device time per step, L2 flushed between steps
+    launches0 = q.qlora_launch_count()
+    q.qlora_timing_begin(32 * args.steps)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        ms = time_steps(wl.step, args.steps, wl.flush, barrier)
+    gemm_ms, gemm_n, gemm_flops = q.qlora_timing_end()
+    launches = q.qlora_launch_count() - launches0
+    q.qlora_check_device_error()
+    ms = max_over_ranks(ms)
+    flops = step_flops() * world
+    value = flops / (ms * 1e-3) / 1e12
+    tokens_per_s = M_TOKENS * world / (ms * 1e-3)
+
+    # end to end through the public API: pinned host inputs -> device -> step -> gradients back to host
+    def e2e_step():
+        wl.h2d()
+        wl.step()
+        wl.d2h()
+    for _ in range(2):
+        e2e_step()
+    ms_e2e = max_over_ranks(time_steps(e2e_step, args.steps, wl.flush, barrier))
+    e2e_value = flops / (ms_e2e * 1e-3) / 1e12
+
+    peak_tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
+                "frac": (achieved / peak_tc) if achieved else None, "traffic": None,
+                "kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05, forward Y and backward dX)",
+                "launches_timed": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1),
+                "peak_kind": f"bf16_tflops_sustained ({peaks['_source']})"}
+    comp = None
+    cpu = None
+    if rank == 0 and world == 1:
+        comp = components(dev, peaks)
+        if not args.no_cpu_baseline:
+            s = OracleSample()
+            times = [s.step() for _ in range(args.cpu_steps)]
+            v = s.flops * len(times) / sum(times) / 1e12
+            cpu = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": s.desc}
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens_per_gpu": M_TOKENS, "small_m": M_SMALL, "r": RANK_R,
+                       "alpha": ALPHA, "weights": "NF4 blk64 + DQ E4M3 blk256", "activations": "bf16",
+                       "l2": "inputs larger than L2; 512 MiB written between timed steps",
+                       "parallelism": f"dp{world}", "step_tflop": flops / 1e12 / world},
+            "tokens_per_s": tokens_per_s,
+            "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": wl.h2d_bytes,
+                    "d2h_bytes_per_step": wl.d2h_bytes, "ms_per_step": ms_e2e},
+            "gpu_launches": launches, "clocks": clk.summary(), "components": comp,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--cpu-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

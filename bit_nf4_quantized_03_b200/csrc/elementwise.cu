@@ -1,0 +1,197 @@
+// Small memory-bound kernels around the tensor-core GEMMs: split reductions
+// of the low-rank products, hi/lo bf16 splitting, gradient finalisation and
+// the SiLU-gated glue between the MLP projections.
+#include "qlora_kernels.h"
+
+namespace qlora {
+
+__device__ __forceinline__ uint16_t f2bf(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+static int blocks_for(int64_t n, int threads) {
+  int64_t g = (n + threads - 1) / threads;
+  if (g > 148 * 32) g = 148 * 32;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+// U (or G) = sum over split partials [split][rows][r_pad], fixed order.
+// Writes any of: fp32 [rows, r]; bf16(scale * U) [rows, r_pad]; hi/lo bf16 [rows, r_pad].
+__global__ void lora_finalize_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
+                                     int r, int r_pad, float scale, float* __restrict__ out_f32,
+                                     uint16_t* __restrict__ out_scaled, uint16_t* __restrict__ out_hi,
+                                     uint16_t* __restrict__ out_lo) {
+  const int64_t total = rows * r_pad;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = idx / r_pad;
+    const int j = static_cast<int>(idx - row * r_pad);
+    float s = 0.f;
+    if (j < r)
+      for (int t = 0; t < splits; ++t) s += part[t * part_stride + idx];
+    if (out_f32 != nullptr && j < r) out_f32[row * r + j] = s;
+    if (out_scaled != nullptr) out_scaled[idx] = f2bf(__fmul_rn(scale, s));
+    if (out_hi != nullptr) {
+      const uint16_t h = f2bf(s);
+      out_hi[idx] = h;
+      out_lo[idx] = f2bf(__fsub_rn(s, bf2f(h)));
+    }
+  }
+}
+
+cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows, int32_t r,
+                                 int32_t r_pad, float scale, float* out_f32, uint16_t* out_scaled_bf16,
+                                 uint16_t* out_hi, uint16_t* out_lo, cudaStream_t st) {
+  const int64_t total = rows * r_pad;
+  lora_finalize_kernel<<<blocks_for(total, 256), 256, 0, st>>>(part, splits, part_stride, rows, r, r_pad, scale,
+                                                                out_f32, out_scaled_bf16, out_hi, out_lo);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+__global__ void split_hilo_kernel(const float* __restrict__ src, int64_t rows, int r, int r_pad,
+                                  uint16_t* __restrict__ hi, uint16_t* __restrict__ lo) {
+  const int64_t total = rows * r_pad;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = idx / r_pad;
+    const int j = static_cast<int>(idx - row * r_pad);
+    const float s = (j < r) ? src[row * r + j] : 0.f;
+    const uint16_t h = f2bf(s);
+    hi[idx] = h;
+    lo[idx] = f2bf(__fsub_rn(s, bf2f(h)));
+  }
+}
+
+cudaError_t launch_split_hilo(const float* src, int64_t rows, int32_t r, int32_t r_pad, uint16_t* hi, uint16_t* lo,
+                              cudaStream_t st) {
+  split_hilo_kernel<<<blocks_for(rows * r_pad, 256), 256, 0, st>>>(src, rows, r, r_pad, hi, lo);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// dB[row, j] (or dA[j, row] when transposed) (+)= scale * sum_t part[t][row][j]
+__global__ void grad_finalize_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
+                                     int r, int ld_part, float scale, float* __restrict__ out, int transpose,
+                                     int accumulate) {
+  const int64_t total = rows * r;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t row, j;
+    if (transpose) {   // consecutive threads walk the contiguous dimension of dA [r, rows]
+      j = idx / rows;
+      row = idx - j * rows;
+    } else {
+      row = idx / r;
+      j = idx - row * r;
+    }
+    float s = 0.f;
+    for (int t = 0; t < splits; ++t) s += part[t * part_stride + row * ld_part + j];
+    s = __fmul_rn(scale, s);
+    const int64_t o = transpose ? (j * rows + row) : (row * r + j);
+    out[o] = accumulate ? (out[o] + s) : s;
+  }
+}
+
+cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_stride, int64_t rows, int32_t r,
+                                 int32_t ld_part, float scale, float* out, int transpose, int accumulate,
+                                 cudaStream_t st) {
+  grad_finalize_kernel<<<blocks_for(rows * r, 256), 256, 0, st>>>(part, splits, part_stride, rows, r, ld_part,
+                                                                   scale, out, transpose, accumulate);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// out[row, col] (+)= sum_t part[t][row][col], 4 columns per thread.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
+                                     int64_t cols, int64_t ld_part, void* __restrict__ out, int out_bf16,
+                                     int accumulate) {
+  const int64_t c4 = cols / 4;
+  const int64_t total = rows * c4;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = idx / c4;
+    const int64_t col = (idx - row * c4) * 4;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = 0; t < splits; ++t) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(part + t * part_stride + row * ld_part + col));
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    if (out_bf16) {
+      uint16_t* o = static_cast<uint16_t*>(out) + row * cols + col;
+      if (accumulate) { s.x += bf2f(o[0]); s.y += bf2f(o[1]); s.z += bf2f(o[2]); s.w += bf2f(o[3]); }
+      uint2 w;
+      w.x = pack_bf16x2(s.x, s.y);
+      w.y = pack_bf16x2(s.z, s.w);
+      *reinterpret_cast<uint2*>(o) = w;
+    } else {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + row * cols + col);
+      if (accumulate) { const float4 y = *o; s.x += y.x; s.y += y.y; s.z += y.z; s.w += y.w; }
+      *o = s;
+    }
+  }
+}
+
+cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_stride, int64_t rows, int64_t cols,
+                                 int64_t ld_part, void* out, int out_bf16, int accumulate, cudaStream_t st) {
+  splitk_reduce_kernel<<<blocks_for(rows * (cols / 4), 256), 256, 0, st>>>(part, splits, part_stride, rows, cols,
+                                                                            ld_part, out, out_bf16, accumulate);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// SiLU-gated glue: h = silu(g) * u ; dg = dh*u*sig*(1 + g*(1-sig)), du = dh*g*sig
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+__global__ void silu_gate_fwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ u,
+                                     uint16_t* __restrict__ h, int64_t count) {
+  const int64_t n8 = count / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 gv = __ldcs(reinterpret_cast<const uint4*>(g) + i);
+    const uint4 uv = __ldcs(reinterpret_cast<const uint4*>(u) + i);
+    const uint32_t ga[4] = {gv.x, gv.y, gv.z, gv.w}, ua[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float g0 = __uint_as_float(ga[t] << 16), g1 = __uint_as_float(ga[t] & 0xFFFF0000u);
+      const float u0 = __uint_as_float(ua[t] << 16), u1 = __uint_as_float(ua[t] & 0xFFFF0000u);
+      o[t] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+    }
+    __stcs(reinterpret_cast<uint4*>(h) + i, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+  for (int64_t i = n8 * 8 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float gg = bf2f(g[i]);
+    h[i] = f2bf(gg * sigmoidf_(gg) * bf2f(u[i]));
+  }
+}
+
+__global__ void silu_gate_bwd_kernel(const uint16_t* __restrict__ dh, const uint16_t* __restrict__ g,
+                                     const uint16_t* __restrict__ u, uint16_t* __restrict__ dg,
+                                     uint16_t* __restrict__ du, int64_t count) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float d = bf2f(dh[i]), gg = bf2f(g[i]), uu = bf2f(u[i]);
+    const float s = sigmoidf_(gg);
+    du[i] = f2bf(d * gg * s);
+    dg[i] = f2bf(d * uu * s * (1.0f + gg * (1.0f - s)));
+  }
+}
+
+cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
+                                 cudaStream_t st) {
+  silu_gate_fwd_kernel<<<blocks_for((count + 7) / 8, 256), 256, 0, st>>>(g, u, h, count);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,
+                                 uint16_t* du, int64_t count, cudaStream_t st) {
+  silu_gate_bwd_kernel<<<blocks_for(count, 256), 256, 0, st>>>(dh, g, u, dg, du, count);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

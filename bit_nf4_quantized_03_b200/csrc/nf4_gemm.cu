@@ -1,0 +1,492 @@
+// Tensor-core GEMM for the frozen-base linear layer and its low-rank branch,
+// sm_100a: TMA-staged operand tiles in 128-byte-swizzled shared memory,
+// tcgen05.mma (kind::f16, BF16 x BF16 -> FP32) accumulating in TMEM, and a
+// persistent, warp-specialised schedule:
+//
+//   warp 0      TMA producer (activation tiles; packed NF4 codes or bf16 B tiles)
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2-5   epilogue: TMEM -> registers -> global (one TMEM lane quarter each)
+//   warps 6-13  (NF4 modes) dequantizers: packed 4-bit codes -> BF16 tile in the
+//               exact shared-memory layout the MMA descriptor expects
+//
+// The NF4 weight is never materialised in BF16 in global memory: each 64-weight
+// block is expanded "right before the GPU multiplies" ("QLoRA: Quantized
+// Low-Rank Adaptation", Piece 2; "Batched 4-bit matmuls"). The low-rank
+// branch rides along as extra K steps into the same accumulator:
+//   forward  Y  = [X | s*U] . [W | B]^T            (U = X A^T)
+//   backward dX = [dY | s*G] . [W ; A]              (G = dY B)
+// Accumulators are double-buffered in TMEM so the epilogue of one tile
+// overlaps the main loop of the next.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "qlora_kernels.h"
+
+namespace qlora {
+
+template <int kBN, int kStages, bool kAMn, int kBMode, bool kExt, bool kHiLo>
+struct GemmCfg {
+  static constexpr int BN = kBN;
+  static constexpr int Stages = kStages;
+  static constexpr bool AMn = kAMn;
+  static constexpr int BMode = kBMode;
+  static constexpr bool Ext = kExt;
+  static constexpr bool HiLo = kHiLo;
+  static constexpr bool Nf4 = (kBMode == kB_Nf4K || kBMode == kB_Nf4MN);
+  static constexpr bool BMn = (kBMode == kB_TmaMN || kBMode == kB_Nf4MN);
+  static constexpr int kABytes = 128 * 64 * 2;
+  static constexpr int kBTile = BN * 64 * 2;
+  static constexpr int kBBytes = kBTile * (HiLo ? 2 : 1);
+  static constexpr int kRBytes = Nf4 ? BN * 32 : 0;
+  static constexpr int kDeqWarps = Nf4 ? 8 : 0;
+  static constexpr int kThreads = (6 + kDeqWarps) * 32;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = Stages * (kABytes + kBBytes + kRBytes) + 1024 + kBarBytes;
+  static_assert(!Nf4 || BN == 256, "dequantizer thread mapping assumes a 256-wide tile");
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM alloc size");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& mb, int& nb, int& split,
+                                            int& kt0, int& nmain, int& next) {
+  split = u % p.splits;
+  const int t = u / p.splits;
+  nb = t % p.tiles_n;
+  mb = t / p.tiles_n;
+  kt0 = split * p.k_per_split;
+  int kt1 = kt0 + p.k_per_split;
+  if (kt1 > p.k_tiles) kt1 = p.k_tiles;
+  nmain = kt1 - kt0;
+  next = (split == 0) ? p.ext_tiles : 0;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Epilogue store of 32 consecutive accumulator columns of one row.
+__device__ __forceinline__ void store_row32(const GemmParams& p, int split, int row, int col0,
+                                            const uint32_t (&v)[32]) {
+  if (row >= p.rows) return;
+  if (p.out_mode == kOutPartial) {
+    float* o = static_cast<float*>(p.out) + split * p.part_stride + static_cast<int64_t>(row) * p.ld_out + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4*>(o + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                                      __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+    return;
+  }
+  const bool full = (col0 + 32 <= p.cols);
+  if (p.out_mode == kOutF32) {
+    float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.ld_out + col0;
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 x = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                               __uint_as_float(v[j + 3]));
+        if (p.accumulate) {
+          const float4 y = *reinterpret_cast<const float4*>(o + j);
+          x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+        }
+        *reinterpret_cast<float4*>(o + j) = x;
+      }
+    } else {
+      for (int j = 0; j < 32 && col0 + j < p.cols; ++j) {
+        float x = __uint_as_float(v[j]);
+        if (p.accumulate) x += o[j];
+        o[j] = x;
+      }
+    }
+    return;
+  }
+  // bf16
+  uint16_t* o = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(row) * p.ld_out + col0;
+  if (full) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      float x[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) x[t] = __uint_as_float(v[j + t]);
+      if (p.accumulate) {
+        const uint4 y = *reinterpret_cast<const uint4*>(o + j);
+        const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          x[2 * t] += __uint_as_float(yy[t] << 16);
+          x[2 * t + 1] += __uint_as_float(yy[t] & 0xFFFF0000u);
+        }
+      }
+      uint4 w;
+      w.x = pack_bf16x2(x[0], x[1]);
+      w.y = pack_bf16x2(x[2], x[3]);
+      w.z = pack_bf16x2(x[4], x[5]);
+      w.w = pack_bf16x2(x[6], x[7]);
+      *reinterpret_cast<uint4*>(o + j) = w;
+    }
+  } else {
+    for (int j = 0; j < 32 && col0 + j < p.cols; ++j) {
+      float x = __uint_as_float(v[j]);
+      if (p.accumulate) x += __uint_as_float(static_cast<uint32_t>(o[j]) << 16);
+      o[j] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+    }
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    qlora_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::Stages * C::kABytes;
+  uint8_t* sR = sB + C::Stages * C::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + C::Stages * C::kRBytes);
+  uint64_t* tma_full = bars;
+  uint64_t* deq_full = bars + C::Stages;
+  uint64_t* empty = bars + 2 * C::Stages;
+  uint64_t* acc_full = bars + 3 * C::Stages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int units = p.tiles_m * p.tiles_n * p.splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::Stages; ++s) {
+      mbar_init(&tma_full[s], 1);
+      mbar_init(&deq_full[s], C::kDeqWarps > 0 ? C::kDeqWarps : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.a);
+      tma_prefetch_desc(&maps.b);
+      if (C::Ext || C::HiLo) tma_prefetch_desc(&maps.b2);
+      if (C::Ext) tma_prefetch_desc(&maps.a2);
+      int stage = 0;
+      uint32_t ph = 0;
+      uint32_t pending = 0;      // stages with a load whose completion nobody has waited for yet
+      uint32_t pend_par = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int mb, nb, split, kt0, nmain, next;
+        decode_unit(p, u, mb, nb, split, kt0, nmain, next);
+        for (int i = 0; i < nmain + next; ++i) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) { ok = false; break; }
+          pending &= ~(1u << stage);
+          uint8_t* a_dst = sA + stage * C::kABytes;
+          uint8_t* b_dst = sB + stage * C::kBBytes;
+          uint64_t* bar = &tma_full[stage];
+          if (i < nmain) {
+            const int kt = kt0 + i;
+            mbar_arrive_expect_tx(bar, C::kABytes + (C::Nf4 ? C::kRBytes : C::kBBytes));
+            if (C::AMn) {
+              tma_load_2d(a_dst, &maps.a, bar, mb * 128, kt * 64);
+              tma_load_2d(a_dst + 8192, &maps.a, bar, mb * 128 + 64, kt * 64);
+            } else {
+              tma_load_2d(a_dst, &maps.a, bar, kt * 64, mb * 128);
+            }
+            if (C::BMode == kB_TmaK) {
+              tma_load_2d(b_dst, &maps.b, bar, kt * 64, nb * C::BN);
+            } else if (C::BMode == kB_TmaMN) {
+#pragma unroll
+              for (int j = 0; j < C::BN / 64; ++j) {
+                tma_load_2d(b_dst + j * 8192, &maps.b, bar, nb * C::BN + 64 * j, kt * 64);
+                if (C::HiLo) tma_load_2d(b_dst + C::kBTile + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, kt * 64);
+              }
+            } else if (C::BMode == kB_Nf4K) {
+              tma_load_2d(sR + stage * C::kRBytes, &maps.b, bar, kt * 32, nb * C::BN);
+            } else {
+              tma_load_2d(sR + stage * C::kRBytes, &maps.b, bar, nb * (C::BN / 2), kt * 64);
+            }
+          } else {
+            const int e = i - nmain;
+            mbar_arrive_expect_tx(bar, C::kABytes + C::kBTile);
+            tma_load_2d(a_dst, &maps.a2, bar, e * 64, mb * 128);
+            if (!C::BMn) {
+              tma_load_2d(b_dst, &maps.b2, bar, e * 64, nb * C::BN);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::BN / 64; ++j)
+                tma_load_2d(b_dst + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, e * 64);
+            }
+          }
+          pending |= (1u << stage);
+          pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
+          if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (ok) {
+        // tail: re-acquire every stage once, so that the MMA's last releases
+        // (asynchronous tcgen05.commit arrivals) have landed before exit
+        for (int s = 0; s < C::Stages; ++s) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) break;
+          if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+        }
+      } else {     // error path: let copies already in flight land before the CTA exits
+        for (int s = 0; s < C::Stages; ++s)
+          if (pending & (1u << s)) mbar_wait(&tma_full[s], (pend_par >> s) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(C::BN, C::AMn, C::BMn);
+      int stage = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int mb, nb, split, kt0, nmain, next;
+        decode_unit(p, u, mb, nb, split, kt0, nmain, next);
+        if (!mbar_wait(&acc_empty[acc], aph ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+        for (int i = 0; i < nmain + next; ++i) {
+          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
+          if (C::Nf4 && !mbar_wait(&deq_full[stage], ph)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = C::AMn ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                       : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = C::BMn ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                       : umma_desc_sw128(b_addr + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            if (C::HiLo) {
+              const uint64_t bd2 = umma_desc_sw128(b_addr + C::kBTile + kk * 2048, 8192, 1024);
+              umma_bf16(d_tmem, ad, bd2, idesc, 1u);
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      int mb, nb, split, kt0, nmain, next;
+      decode_unit(p, u, mb, nb, split, kt0, nmain, next);
+      if (!mbar_wait(&acc_full[acc], aph)) break;
+      tc_fence_after();
+      const int row = mb * 128 + q * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+#pragma unroll 1
+      for (int c = 0; c < C::BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, v);
+        tmem_ld_wait();
+        store_row32(p, split, row, nb * C::BN + c * 32, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  } else if (C::Nf4) {
+    // ------------------------------------------------------------ dequantizers
+    const int dt = threadIdx.x - 192;           // 0..255
+    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
+    // K-major (forward): thread = W row inside the 256-row tile.
+    // MN-major (backward): thread = (W row i of the 64-row K step, 64-col chunk c).
+    const int i_mn = dt & 63;
+    const int c_mn = dt >> 6;
+    const int srow = (C::BMode == kB_Nf4K) ? dt : i_mn;     // row whose 128-B line we write
+    const int sw = srow & 7;
+    const uint32_t r_off = (C::BMode == kB_Nf4K) ? static_cast<uint32_t>(dt * 32)
+                                                 : static_cast<uint32_t>(i_mn * (C::BN / 2) + c_mn * 32);
+    const uint32_t b_off = (C::BMode == kB_Nf4K)
+                               ? static_cast<uint32_t>((dt >> 3) * 1024 + (dt & 7) * 128)
+                               : static_cast<uint32_t>(c_mn * 8192 + (i_mn >> 3) * 1024 + (i_mn & 7) * 128);
+    int stage = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int mb, nb, split, kt0, nmain, next;
+      decode_unit(p, u, mb, nb, split, kt0, nmain, next);
+      for (int i = 0; i < nmain + next; ++i) {
+        if (i < nmain) {
+          const int kt = kt0 + i;
+          int64_t wrow, kb;
+          if (C::BMode == kB_Nf4K) { wrow = static_cast<int64_t>(nb) * C::BN + dt; kb = kt; }
+          else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(nb) * (C::BN / 64) + c_mn; }
+          const bool valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
+          const float c = valid ? block_scale(p.scales, wrow * p.w_kblocks + kb, mean) : 0.f;
+          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
+          const uint32_t bdst = smem_u32(sB + stage * C::kBBytes) + b_off;
+          if (valid) {
+            const uint32_t rsrc = smem_u32(sR + stage * C::kRBytes) + r_off;
+            const uint4 w0 = ld_shared_v4(rsrc);
+            const uint4 w1 = ld_shared_v4(rsrc + 16);
+            const Nf4Lut lut = nf4_build_lut(p.tab, c);
+            st_shared_v4(bdst + ((0 ^ sw) << 4), nf4_lookup8(lut, w0.x));
+            st_shared_v4(bdst + ((1 ^ sw) << 4), nf4_lookup8(lut, w0.y));
+            st_shared_v4(bdst + ((2 ^ sw) << 4), nf4_lookup8(lut, w0.z));
+            st_shared_v4(bdst + ((3 ^ sw) << 4), nf4_lookup8(lut, w0.w));
+            st_shared_v4(bdst + ((4 ^ sw) << 4), nf4_lookup8(lut, w1.x));
+            st_shared_v4(bdst + ((5 ^ sw) << 4), nf4_lookup8(lut, w1.y));
+            st_shared_v4(bdst + ((6 ^ sw) << 4), nf4_lookup8(lut, w1.z));
+            st_shared_v4(bdst + ((7 ^ sw) << 4), nf4_lookup8(lut, w1.w));
+          } else {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) st_shared_v4(bdst + (j << 4), z);
+          }
+          fence_proxy_async_smem();
+        } else {
+          // extension step: the producer loads the tile; only keep the phases in step
+          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&deq_full[stage]);
+        if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <class C>
+static cudaError_t launch_cfg(const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(qlora_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
+  qlora_gemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p, maps);
+  return cudaGetLastError();
+}
+
+using CfgFwd = GemmCfg<256, 4, false, kB_Nf4K, true, false>;
+using CfgBwd = GemmCfg<256, 4, false, kB_Nf4MN, true, false>;
+using CfgDownK = GemmCfg<64, 6, false, kB_TmaK, false, false>;
+using CfgDownMN = GemmCfg<64, 6, false, kB_TmaMN, false, false>;
+using CfgGrad = GemmCfg<64, 6, true, kB_TmaMN, false, true>;
+using CfgDownK128 = GemmCfg<128, 5, false, kB_TmaK, false, false>;
+using CfgDownMN128 = GemmCfg<128, 5, false, kB_TmaMN, false, false>;
+using CfgGrad128 = GemmCfg<128, 4, true, kB_TmaMN, false, true>;
+
+int gemm_bn(GemmKind kind) {
+  switch (kind) {
+    case kGemmFwd: case kGemmBwdDx: return 256;
+    case kGemmLoraDownK128: case kGemmLoraDownMN128: case kGemmLoraGrad128: return 128;
+    default: return 64;
+  }
+}
+
+static cudaError_t launch_gemm_impl(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid,
+                                    cudaStream_t st) {
+  switch (kind) {
+    case kGemmFwd: return launch_cfg<CfgFwd>(p, maps, grid, st);
+    case kGemmBwdDx: return launch_cfg<CfgBwd>(p, maps, grid, st);
+    case kGemmLoraDownK: return launch_cfg<CfgDownK>(p, maps, grid, st);
+    case kGemmLoraDownMN: return launch_cfg<CfgDownMN>(p, maps, grid, st);
+    case kGemmLoraGrad: return launch_cfg<CfgGrad>(p, maps, grid, st);
+    case kGemmLoraDownK128: return launch_cfg<CfgDownK128>(p, maps, grid, st);
+    case kGemmLoraDownMN128: return launch_cfg<CfgDownMN128>(p, maps, grid, st);
+    case kGemmLoraGrad128: return launch_cfg<CfgGrad128>(p, maps, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st,
+                        double algo_flops) {
+  const bool timed = (kind == kGemmFwd || kind == kGemmBwdDx) && timing_active();
+  if (timed) timing_record(st, true, algo_flops);
+  const cudaError_t e = launch_gemm_impl(kind, p, maps, grid, st);
+  if (timed) timing_record(st, false, algo_flops);
+  count_launches(1);
+  return e;
+}
+
+}  // namespace qlora

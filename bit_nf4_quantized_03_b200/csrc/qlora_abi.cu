@@ -1,0 +1,537 @@
+// C ABI of libqlora: argument checks, the NF4 level table, workspace planning
+// and the launch sequence of each entry point. See include/qlora.h.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/qlora.h"
+#include "qlora_kernels.h"
+
+using namespace qlora;
+
+// ---------------------------------------------------------------------------
+// Launch accounting and the optional device-time hook for the fused GEMMs.
+// ---------------------------------------------------------------------------
+namespace qlora {
+namespace {
+std::atomic<int64_t> g_launches{0};
+std::atomic<bool> g_timing_on{false};
+std::mutex g_timing_mu;
+std::vector<cudaEvent_t> g_events;     // pairs: start, stop
+std::vector<double> g_event_flops;
+size_t g_events_used = 0;
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+bool timing_active() { return g_timing_on.load(std::memory_order_relaxed); }
+
+void timing_record(cudaStream_t st, bool start, double flops) {
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  if (!g_timing_on) return;
+  if (start) {
+    if (g_events_used + 2 > g_events.size()) return;
+    cudaEventRecord(g_events[g_events_used], st);
+    g_event_flops[g_events_used / 2] = flops;
+  } else {
+    if (g_events_used + 2 > g_events.size()) return;
+    cudaEventRecord(g_events[g_events_used + 1], st);
+    g_events_used += 2;
+  }
+}
+}  // namespace qlora
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// NF4 levels: 16 quantiles of the standard normal distribution with an exact
+// zero, normalised to [-1, 1] ("QLoRA Explained", "4-Bit NormalFloat (NF4)
+// Quantization"; "QLoRA: Quantized Low-Rank Adaptation", "NF4: a 4-bit format
+// matched to weight statistics"). Construction: 8 positive quantiles at
+// probabilities equally spaced from delta to 1/2 (1/2 itself dropped), 7
+// negative quantiles the same way on 8 points, and 0; divided by the largest.
+// delta = ((1 - 1/30) + (1 - 1/32)) / 2 keeps the outermost quantile finite.
+// The inverse CDF is found here by Newton's method on erfc.
+// ---------------------------------------------------------------------------
+double normal_quantile(double p) {
+  const double inv_sqrt2 = 0.70710678118654752440;
+  const double inv_sqrt2pi = 0.39894228040143267794;
+  double x = 0.0;
+  for (int it = 0; it < 100; ++it) {
+    const double cdf = 0.5 * std::erfc(-x * inv_sqrt2);
+    const double pdf = inv_sqrt2pi * std::exp(-0.5 * x * x);
+    const double dx = (cdf - p) / pdf;
+    x -= dx;
+    if (std::fabs(dx) < 1e-17 * (1.0 + std::fabs(x))) break;
+  }
+  return x;
+}
+
+Nf4Table build_table() {
+  const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+  double v[16];
+  int n = 0;
+  const double step9 = (0.5 - delta) / 8.0;   // 9 points delta..0.5
+  const double step8 = (0.5 - delta) / 7.0;   // 8 points delta..0.5
+  double pos[8], neg[7];
+  for (int i = 0; i < 8; ++i) pos[i] = normal_quantile(i * step9 + delta);
+  for (int i = 0; i < 7; ++i) neg[i] = -normal_quantile(i * step8 + delta);
+  for (int i = 0; i < 7; ++i) v[n++] = neg[i];       // ascending: most negative first
+  v[n++] = 0.0;
+  for (int i = 7; i >= 0; --i) v[n++] = pos[i];
+  const double vmax = pos[0];
+  Nf4Table t;
+  for (int i = 0; i < 16; ++i) t.lv[i] = static_cast<float>(v[i] / vmax);
+  for (int i = 0; i < 15; ++i) t.mid[i] = (t.lv[i] + t.lv[i + 1]) * 0.5f;
+  t.mid[15] = 2.0f;
+  return t;
+}
+
+const Nf4Table& table() {
+  static const Nf4Table t = build_table();
+  return t;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool weight_ok(const qlora_nf4_weight* w) {
+  if (w == nullptr || w->n < 1 || w->k < 1) return false;
+  if (w->blocksize != QLORA_BLOCKSIZE || w->dq_blocksize != QLORA_DQ_BLOCKSIZE) return false;
+  if (w->codes == nullptr || !aligned16(w->codes)) return false;
+  if (w->mode == QLORA_SCALE_BF16) return w->scale_bf16 != nullptr && aligned16(w->scale_bf16);
+  if (w->mode == QLORA_SCALE_DQ_FP8)
+    return w->scale_fp8 != nullptr && w->dq_scale != nullptr && w->dq_mean != nullptr && aligned16(w->scale_fp8) &&
+           aligned16(w->dq_scale);
+  return false;
+}
+
+ScaleSrc scale_src(const qlora_nf4_weight* w) {
+  ScaleSrc s{};
+  if (w->mode == QLORA_SCALE_BF16) {
+    s.bf16 = w->scale_bf16;
+  } else {
+    s.fp8 = w->scale_fp8;
+    s.dq_scale = w->dq_scale;
+    s.dq_mean = w->dq_mean;
+  }
+  return s;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------
+// Linear-layer plan: split counts and workspace carve-up. Deterministic in
+// (m, n, k, r, SM count) so the size query and the call always agree.
+// ---------------------------------------------------------------------------
+struct Split {
+  int splits = 1, kps = 1;
+};
+
+Split choose_split(int64_t tiles, int64_t k_tiles, int sms) {
+  Split s;
+  int64_t want = std::max<int64_t>(1, sms / std::max<int64_t>(tiles, 1));
+  want = std::min<int64_t>(want, std::max<int64_t>(k_tiles, 1));
+  want = std::min<int64_t>(want, 64);
+  s.kps = static_cast<int>(cdiv(std::max<int64_t>(k_tiles, 1), want));
+  s.splits = static_cast<int>(cdiv(std::max<int64_t>(k_tiles, 1), s.kps));
+  return s;
+}
+
+struct Plan {
+  int r_pad = 64;
+  GemmKind down_k = kGemmLoraDownK, down_mn = kGemmLoraDownMN, grad = kGemmLoraGrad;
+  Split u, g, db, da, fwd;
+  size_t off_u32 = 0, off_scaled = 0, off_hi_a = 0, off_lo_a = 0, off_hi_b = 0, off_lo_b = 0, off_part = 0,
+         total = 0;
+};
+
+Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
+  Plan P;
+  const int sms = num_sms();
+  P.r_pad = (r <= 64) ? 64 : 128;
+  if (P.r_pad == 128) {
+    P.down_k = kGemmLoraDownK128;
+    P.down_mn = kGemmLoraDownMN128;
+    P.grad = kGemmLoraGrad128;
+  }
+  const int64_t tm = cdiv(m, 128);
+  P.u = choose_split(tm, k / 64, sms);
+  P.g = choose_split(tm, cdiv(n, 64), sms);
+  P.db = choose_split(cdiv(n, 128), cdiv(m, 64), sms);
+  P.da = choose_split(cdiv(k, 128), cdiv(m, 64), sms);
+  const int64_t fwd_tiles = tm * cdiv(n, 256);
+  if (fwd_tiles * 2 <= sms) P.fwd = choose_split(fwd_tiles, k / 64, sms);
+  const size_t rp = static_cast<size_t>(P.r_pad);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  P.off_u32 = take(static_cast<size_t>(m) * r * 4);
+  P.off_scaled = take(static_cast<size_t>(m) * rp * 2);
+  P.off_hi_a = take(static_cast<size_t>(m) * rp * 2);
+  P.off_lo_a = take(static_cast<size_t>(m) * rp * 2);
+  P.off_hi_b = take(static_cast<size_t>(m) * rp * 2);
+  P.off_lo_b = take(static_cast<size_t>(m) * rp * 2);
+  size_t part = 0;
+  part = std::max(part, static_cast<size_t>(P.u.splits) * m * rp);
+  part = std::max(part, static_cast<size_t>(P.g.splits) * m * rp);
+  part = std::max(part, static_cast<size_t>(P.db.splits) * n * rp);
+  part = std::max(part, static_cast<size_t>(P.da.splits) * k * rp);
+  if (P.fwd.splits > 1) part = std::max(part, static_cast<size_t>(P.fwd.splits) * m * cdiv(n, 256) * 256);
+  P.off_part = take(part * 4);
+  P.total = off;
+  return P;
+}
+
+bool linear_args_ok(const qlora_nf4_weight* w, const void* X, int64_t m, const void* A, const void* B, int32_t r) {
+  if (!weight_ok(w) || X == nullptr || A == nullptr || B == nullptr) return false;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return false;
+  if (m < 1 || m > (int64_t(1) << 31) - 1) return false;
+  if (w->n > (int64_t(1) << 31) - 1 || w->k > (int64_t(1) << 31) - 1) return false;
+  return true;
+}
+
+int linear_shape_status(const qlora_nf4_weight* w, int32_t r) {
+  if (w->k % 64 != 0 || w->n % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (!(r == 8 || r == 16 || r == 32 || r == 64 || r == 128)) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+GemmParams base_params(int64_t rows, int64_t cols, int bn, int64_t k_tiles, Split sp) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.rows = static_cast<int32_t>(rows);
+  p.cols = static_cast<int32_t>(cols);
+  p.tiles_m = static_cast<int32_t>(cdiv(rows, 128));
+  p.tiles_n = static_cast<int32_t>(cdiv(cols, bn));
+  p.k_tiles = static_cast<int32_t>(k_tiles);
+  // one split covers the whole reduction
+  p.splits = sp.splits > 1 ? sp.splits : 1;
+  p.k_per_split = sp.splits > 1 ? sp.kps : static_cast<int32_t>(k_tiles);
+  p.tab = table();
+  return p;
+}
+
+int grid_of(const GemmParams& p) {
+  const int64_t units = static_cast<int64_t>(p.tiles_m) * p.tiles_n * p.splits;
+  return static_cast<int>(std::min<int64_t>(units, num_sms()));
+}
+
+const CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+const CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+
+// bf16 matrix [rows, cols] row-major, 128-B swizzled boxes of [64 cols, box_rows].
+bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  return tmap_2d(m, base, kBF16, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                 static_cast<uint64_t>(cols) * 2, 64, box_rows, true);
+}
+
+// Low-rank product U (or G): partial GEMM over the reduction, then finalize.
+int run_lora_down(const Plan& P, bool b_mn, const uint16_t* act, int64_t m, int64_t red, const uint16_t* adapter,
+                  int32_t r, float scale, char* ws, float* out_f32, uint16_t* out_scaled, uint16_t* out_hi,
+                  uint16_t* out_lo, cudaStream_t st) {
+  const Split sp = b_mn ? P.g : P.u;
+  GemmParams p = base_params(m, P.r_pad, P.r_pad, b_mn ? cdiv(red, 64) : red / 64, sp);
+  p.out = ws + P.off_part;
+  p.ld_out = P.r_pad;
+  p.part_stride = m * P.r_pad;
+  p.out_mode = kOutPartial;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  bool ok = map_bf16(&maps.a, act, m, red, 128);
+  if (!b_mn) {  // adapter A [r, red] is K-major
+    ok = ok && tmap_2d(&maps.b, adapter, kBF16, red, r, red * 2, 64, P.r_pad, true);
+  } else {      // adapter B [red, r] is MN-major (r contiguous)
+    ok = ok && tmap_2d(&maps.b, adapter, kBF16, r, red, r * 2, 64, 64, true);
+  }
+  if (!ok) return QLORA_ERR_CUDA;
+  cudaError_t e = launch_gemm(b_mn ? P.down_mn : P.down_k, p, maps, grid_of(p), st);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  e = launch_lora_finalize(static_cast<const float*>(p.out), sp.splits, p.part_stride, m, r, P.r_pad, scale,
+                           out_f32, out_scaled, out_hi, out_lo, st);
+  return cuda_status(e);
+}
+
+// dB (rows = n, act = dY) or dA^T (rows = k, act = X): sum over tokens of act^T . [hi + lo].
+int run_lora_grad(const Plan& P, const Split& sp, const uint16_t* act, int64_t m, int64_t rows, const uint16_t* hi,
+                  const uint16_t* lo, int32_t r, float scale, float* out, int transpose, int accumulate, char* ws,
+                  cudaStream_t st) {
+  GemmParams p = base_params(rows, P.r_pad, P.r_pad, cdiv(m, 64), sp);
+  p.out = ws + P.off_part;
+  p.ld_out = P.r_pad;
+  p.part_stride = rows * P.r_pad;
+  p.out_mode = kOutPartial;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  bool ok = tmap_2d(&maps.a, act, kBF16, rows, m, rows * 2, 64, 64, true);          // [m, rows], MN-major A
+  ok = ok && tmap_2d(&maps.b, hi, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, true);    // [m, r_pad], MN-major B
+  ok = ok && tmap_2d(&maps.b2, lo, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, true);
+  if (!ok) return QLORA_ERR_CUDA;
+  cudaError_t e = launch_gemm(P.grad, p, maps, grid_of(p), st);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  e = launch_grad_finalize(static_cast<const float*>(p.out), sp.splits, p.part_stride, rows, r, P.r_pad, scale, out,
+                           transpose, accumulate, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qlora_status_string(int s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID: return "invalid argument";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_DEVICE: return "a kernel gave up on a bounded wait";
+    default: return "unknown status";
+  }
+}
+
+const char* qlora_version(void) { return "qlora-nf4-b200 0.1 (sm_100a)"; }
+
+int qlora_nf4_levels(float levels[16], float mid[15]) {
+  const Nf4Table& t = table();
+  if (levels != nullptr) std::memcpy(levels, t.lv, sizeof(float) * 16);
+  if (mid != nullptr) std::memcpy(mid, t.mid, sizeof(float) * 15);
+  return QLORA_OK;
+}
+
+size_t qlora_nf4_quantize_workspace_bytes(int64_t n, int64_t k, int32_t mode) {
+  if (mode != QLORA_SCALE_DQ_FP8 || n < 1 || k < 1) return 0;
+  return quant_ws_layout(n * k).total;
+}
+
+int qlora_nf4_quantize(const float* W, qlora_nf4_weight* w, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (W == nullptr || !aligned16(W) || !weight_ok(w)) return QLORA_ERR_INVALID;
+  const int64_t n_elem = w->n * w->k;
+  const bool dq = (w->mode == QLORA_SCALE_DQ_FP8);
+  if (dq) {
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < quant_ws_layout(n_elem).total) return QLORA_ERR_WORKSPACE;
+  }
+  const cudaError_t e =
+      launch_quantize(W, n_elem, table(), w->codes, dq ? nullptr : w->scale_bf16, dq ? w->scale_fp8 : nullptr,
+                      dq ? w->dq_scale : nullptr, dq ? w->dq_mean : nullptr, ws, num_sms(),
+                      reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+int qlora_nf4_dequantize(const qlora_nf4_weight* w, uint16_t* out_bf16, qlora_stream_t stream) {
+  if (!weight_ok(w) || out_bf16 == nullptr || !aligned16(out_bf16)) return QLORA_ERR_INVALID;
+  const cudaError_t e = launch_dequantize(w->codes, scale_src(w), w->n * w->k, table(), out_bf16, num_sms(),
+                                          reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+size_t qlora_linear_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) {
+  if (m < 1 || n < 1 || k < 1 || r < 1 || r > 128) return 0;
+  return make_plan(m, n, k, r).total;
+}
+
+int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, const uint16_t* A, const uint16_t* B,
+                     int32_t r, float alpha, void* Y, int32_t y_dtype, float* U_save, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream) {
+  if (!linear_args_ok(w, X, m, A, B, r) || Y == nullptr || !aligned16(Y)) return QLORA_ERR_INVALID;
+  if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_FP32) return QLORA_ERR_INVALID;
+  if (U_save != nullptr && !aligned16(U_save)) return QLORA_ERR_INVALID;
+  const int sst = linear_shape_status(w, r);
+  if (sst != QLORA_OK) return sst;
+  const int64_t n = w->n, k = w->k;
+  const Plan P = make_plan(m, n, k, r);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < P.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* wsb = static_cast<char*>(ws);
+  const float s = alpha / static_cast<float>(r);
+  uint16_t* sU = reinterpret_cast<uint16_t*>(wsb + P.off_scaled);
+
+  // U = X A^T (fp32, optionally saved) and bf16(s * U) for the K extension
+  int rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st);
+  if (rc != QLORA_OK) return rc;
+
+  GemmParams p = base_params(m, n, 256, k / 64, P.fwd);
+  p.ext_tiles = P.r_pad / 64;
+  p.scales = scale_src(w);
+  p.w_kblocks = k / 64;
+  p.w_rows = static_cast<int32_t>(n);
+  if (P.fwd.splits > 1) {
+    p.out = wsb + P.off_part;
+    p.ld_out = static_cast<int64_t>(p.tiles_n) * 256;
+    p.part_stride = m * p.ld_out;
+    p.out_mode = kOutPartial;
+  } else {
+    p.out = Y;
+    p.ld_out = n;
+    p.out_mode = (y_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
+  }
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  bool ok = map_bf16(&maps.a, X, m, k, 128);
+  ok = ok && tmap_2d(&maps.b, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                     static_cast<uint64_t>(k / 2), 32, 256, false);
+  ok = ok && map_bf16(&maps.a2, sU, m, P.r_pad, 128);
+  ok = ok && tmap_2d(&maps.b2, B, kBF16, r, n, r * 2, 64, 256, true);
+  if (!ok) return QLORA_ERR_CUDA;
+  const double fwd_flops = 2.0 * double(m) * double(n) * double(k + r);
+  cudaError_t e = launch_gemm(kGemmFwd, p, maps, grid_of(p), st, fwd_flops);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  if (P.fwd.splits > 1) {
+    e = launch_splitk_reduce(static_cast<const float*>(p.out), P.fwd.splits, p.part_stride, m, n, p.ld_out, Y,
+                             y_dtype == QLORA_DTYPE_BF16, 0, st);
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
+int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t m, const uint16_t* A,
+                     const uint16_t* B, int32_t r, float alpha, const float* U_saved, void* dX, int32_t dx_dtype,
+                     float* dA, float* dB, int32_t flags, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!linear_args_ok(w, X, m, A, B, r) || dY == nullptr || !aligned16(dY)) return QLORA_ERR_INVALID;
+  if (dA == nullptr || dB == nullptr || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_INVALID;
+  if (dX != nullptr && (!aligned16(dX) || (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_FP32)))
+    return QLORA_ERR_INVALID;
+  if (U_saved != nullptr && !aligned16(U_saved)) return QLORA_ERR_INVALID;
+  if ((flags & ~(QLORA_BWD_ACCUMULATE_GRADS | QLORA_BWD_ACCUMULATE_DX)) != 0) return QLORA_ERR_INVALID;
+  const int sst = linear_shape_status(w, r);
+  if (sst != QLORA_OK) return sst;
+  const int64_t n = w->n, k = w->k;
+  const Plan P = make_plan(m, n, k, r);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < P.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* wsb = static_cast<char*>(ws);
+  const float s = alpha / static_cast<float>(r);
+  uint16_t* sG = reinterpret_cast<uint16_t*>(wsb + P.off_scaled);
+  uint16_t* g_hi = reinterpret_cast<uint16_t*>(wsb + P.off_hi_b);
+  uint16_t* g_lo = reinterpret_cast<uint16_t*>(wsb + P.off_lo_b);
+  uint16_t* u_hi = reinterpret_cast<uint16_t*>(wsb + P.off_hi_a);
+  uint16_t* u_lo = reinterpret_cast<uint16_t*>(wsb + P.off_lo_a);
+  const int acc_grads = (flags & QLORA_BWD_ACCUMULATE_GRADS) ? 1 : 0;
+
+  // G = dY B: bf16(s G) for the dX extension, hi/lo bf16 for dA
+  int rc = run_lora_down(P, true, dY, m, n, B, r, s, wsb, nullptr, sG, g_hi, g_lo, st);
+  if (rc != QLORA_OK) return rc;
+  // U = X A^T as hi/lo bf16 for dB (recomputed when not saved)
+  if (U_saved != nullptr) {
+    if (launch_split_hilo(U_saved, m, r, P.r_pad, u_hi, u_lo, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  } else {
+    rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, nullptr, nullptr, u_hi, u_lo, st);
+    if (rc != QLORA_OK) return rc;
+  }
+
+  if (dX != nullptr) {
+    GemmParams p = base_params(m, k, 256, cdiv(n, 64), Split{});
+    p.ext_tiles = P.r_pad / 64;
+    p.scales = scale_src(w);
+    p.w_kblocks = k / 64;
+    p.w_rows = static_cast<int32_t>(n);
+    p.out = dX;
+    p.ld_out = k;
+    p.out_mode = (dx_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
+    p.accumulate = (flags & QLORA_BWD_ACCUMULATE_DX) ? 1 : 0;
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    bool ok = map_bf16(&maps.a, dY, m, n, 128);
+    ok = ok && tmap_2d(&maps.b, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                       static_cast<uint64_t>(k / 2), 128, 64, false);
+    ok = ok && map_bf16(&maps.a2, sG, m, P.r_pad, 128);
+    ok = ok && tmap_2d(&maps.b2, A, kBF16, k, r, k * 2, 64, 64, true);
+    if (!ok) return QLORA_ERR_CUDA;
+    const double dx_flops = 2.0 * double(m) * double(k) * double(n + r);
+    if (launch_gemm(kGemmBwdDx, p, maps, grid_of(p), st, dx_flops) != cudaSuccess) return QLORA_ERR_CUDA;
+  }
+
+  rc = run_lora_grad(P, P.db, dY, m, n, u_hi, u_lo, r, s, dB, 0, acc_grads, wsb, st);
+  if (rc != QLORA_OK) return rc;
+  rc = run_lora_grad(P, P.da, X, m, k, g_hi, g_lo, r, s, dA, 1, acc_grads, wsb, st);
+  return rc;
+}
+
+int qlora_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count, qlora_stream_t stream) {
+  if (count < 0) return QLORA_ERR_INVALID;
+  if (count == 0) return QLORA_OK;
+  if (g == nullptr || u == nullptr || h == nullptr || !aligned16(g) || !aligned16(u) || !aligned16(h))
+    return QLORA_ERR_INVALID;
+  return cuda_status(launch_silu_gate_fwd(g, u, h, count, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg, uint16_t* du,
+                        int64_t count, qlora_stream_t stream) {
+  if (count < 0) return QLORA_ERR_INVALID;
+  if (count == 0) return QLORA_OK;
+  if (dh == nullptr || g == nullptr || u == nullptr || dg == nullptr || du == nullptr) return QLORA_ERR_INVALID;
+  return cuda_status(launch_silu_gate_bwd(dh, g, u, dg, du, count, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int64_t qlora_launch_count(void) { return qlora::g_launches.load(); }
+
+int qlora_timing_begin(int32_t max_launches) {
+  if (max_launches < 1) return QLORA_ERR_INVALID;
+  std::lock_guard<std::mutex> g(qlora::g_timing_mu);
+  for (cudaEvent_t ev : qlora::g_events) cudaEventDestroy(ev);
+  qlora::g_events.assign(static_cast<size_t>(max_launches) * 2, nullptr);
+  qlora::g_event_flops.assign(static_cast<size_t>(max_launches), 0.0);
+  for (auto& ev : qlora::g_events)
+    if (cudaEventCreate(&ev) != cudaSuccess) return QLORA_ERR_CUDA;
+  qlora::g_events_used = 0;
+  qlora::g_timing_on = true;
+  return QLORA_OK;
+}
+
+int qlora_timing_end(double* total_ms, int32_t* launches, double* flops) {
+  std::lock_guard<std::mutex> g(qlora::g_timing_mu);
+  qlora::g_timing_on = false;
+  double ms = 0.0, fl = 0.0;
+  int rc = QLORA_OK;
+  for (size_t i = 0; i + 1 < qlora::g_events_used; i += 2) {
+    float t = 0.f;
+    if (cudaEventSynchronize(qlora::g_events[i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, qlora::g_events[i], qlora::g_events[i + 1]) != cudaSuccess) {
+      rc = QLORA_ERR_CUDA;
+      break;
+    }
+    ms += t;
+    fl += qlora::g_event_flops[i / 2];
+  }
+  if (total_ms) *total_ms = ms;
+  if (launches) *launches = static_cast<int32_t>(qlora::g_events_used / 2);
+  if (flops) *flops = fl;
+  for (cudaEvent_t ev : qlora::g_events) cudaEventDestroy(ev);
+  qlora::g_events.clear();
+  qlora::g_event_flops.clear();
+  qlora::g_events_used = 0;
+  return rc;
+}
+
+int qlora_check_device_error(qlora_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, qlora::g_device_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(qlora::g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_ERR_DEVICE;
+  }
+  return QLORA_OK;
+}
+
+}  // extern "C"

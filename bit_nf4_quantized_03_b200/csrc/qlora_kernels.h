@@ -1,0 +1,121 @@
+// Internal launch interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qlora_device.cuh"
+
+namespace qlora {
+
+// ----------------------------------------------------------------- quantize
+struct QuantWsLayout {
+  size_t absmax_off, part_a_off, part_b_off, mean_off, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline QuantWsLayout quant_ws_layout(int64_t n_elem) {
+  const int64_t nblk = (n_elem + 63) / 64;
+  const int64_t pa = (nblk + 511) / 512;
+  const int64_t pb = (pa + 511) / 512 + 1;
+  QuantWsLayout L;
+  L.absmax_off = 0;
+  L.part_a_off = align_up(static_cast<size_t>(nblk) * 4, 256);
+  L.part_b_off = L.part_a_off + align_up(static_cast<size_t>(pa) * 8, 256);
+  L.mean_off = L.part_b_off + align_up(static_cast<size_t>(pb) * 8, 256);
+  L.total = L.mean_off + 256;
+  return L;
+}
+
+cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab, uint8_t* codes,
+                            uint16_t* scale_bf16, uint8_t* scale_fp8, float* dq_scale, float* dq_mean,
+                            void* ws, int num_sms, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t n_elem, const Nf4Table& tab,
+                              uint16_t* out, int num_sms, cudaStream_t st);
+
+// --------------------------------------------------------------------- GEMM
+// Operand sources of the tensor-core GEMM D[rows, cols] = sum_k A[row, k] B[col, k].
+enum BMode : int {
+  kB_TmaK = 0,    // bf16 [cols, K] row-major via TMA (K-major)
+  kB_TmaMN = 1,   // bf16 [K, cols] row-major via TMA (MN-major)
+  kB_Nf4K = 2,    // NF4 weight W[cols, K], dequantized in shared memory (forward)
+  kB_Nf4MN = 3,   // NF4 weight W[K, cols], dequantized in shared memory (backward dX)
+};
+
+enum OutMode : int {
+  kOutBF16 = 0,     // bf16 [rows, cols] with leading dimension ld_out
+  kOutF32 = 1,      // fp32 [rows, cols]
+  kOutPartial = 2,  // fp32 split-K partial: out + split * part_stride, [rows, ld_out]
+};
+
+struct GemmParams {
+  int32_t rows, cols;          // problem size of D
+  int32_t tiles_m, tiles_n;    // 128-row and BN-col tiles
+  int32_t k_tiles;             // main-loop 64-wide K steps
+  int32_t ext_tiles;           // extra K steps from the second operand pair (low-rank branch)
+  int32_t splits, k_per_split; // split of the main K steps
+  // NF4 operand
+  ScaleSrc scales;
+  int64_t w_kblocks;           // 64-blocks per row of W
+  int32_t w_rows;              // rows of W
+  // output
+  void* out;
+  int64_t ld_out;
+  int64_t part_stride;         // elements between split partials
+  int32_t out_mode;
+  int32_t accumulate;          // kOutBF16/kOutF32: out += D
+  Nf4Table tab;
+};
+
+struct GemmMaps {
+  CUtensorMap a, b, a2, b2;    // b = codes for NF4 modes; b2 = lo half for hi/lo mode
+};
+
+// Host helpers (nf4_gemm.cu)
+bool tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+// Launch variants
+enum GemmKind : int {
+  kGemmFwd = 0,        // A = X (K-major), B = NF4 K-major, ext: [s*U | B_lora]
+  kGemmBwdDx = 1,      // A = dY (K-major), B = NF4 MN-major, ext: [s*G | A_lora]
+  kGemmLoraDownK = 2,  // A K-major, B K-major, BN = 64 (U = X A^T)
+  kGemmLoraDownMN = 3, // A K-major, B MN-major, BN = 64 (G = dY B)
+  kGemmLoraGrad = 4,   // A MN-major, B MN-major hi+lo, BN = 64 (dB, dA^T)
+  kGemmLoraDownK128 = 5,
+  kGemmLoraDownMN128 = 6,
+  kGemmLoraGrad128 = 7,
+};
+
+int gemm_bn(GemmKind kind);
+// algo_flops: algorithmic flops of this launch, used only by the optional timing hook
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st,
+                        double algo_flops = 0.0);
+
+// Launch accounting (qlora_abi.cu): every kernel launch is counted; fused NF4
+// GEMM launches can additionally be bracketed by timing events.
+void count_launches(int n);
+bool timing_active();
+void timing_record(cudaStream_t st, bool start, double flops);
+
+// ------------------------------------------------------------- elementwise
+cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
+                                 int32_t r, int32_t r_pad, float scale, float* out_f32,
+                                 uint16_t* out_scaled_bf16, uint16_t* out_hi, uint16_t* out_lo,
+                                 cudaStream_t st);
+cudaError_t launch_split_hilo(const float* src, int64_t rows, int32_t r, int32_t r_pad, uint16_t* hi,
+                              uint16_t* lo, cudaStream_t st);
+cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
+                                 int32_t r, int32_t ld_part, float scale, float* out, int transpose,
+                                 int accumulate, cudaStream_t st);
+cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_stride, int64_t rows,
+                                 int64_t cols, int64_t ld_part, void* out, int out_bf16, int accumulate,
+                                 cudaStream_t st);
+cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
+                                 cudaStream_t st);
+cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,
+                                 uint16_t* du, int64_t count, cudaStream_t st);
+
+}  // namespace qlora

@@ -1,0 +1,199 @@
+/*
+ * qlora.h -- C ABI of libqlora: the frozen-base linear layer of QLoRA on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes (sources are web pages on QLoRA, cited by title/section):
+ *
+ *  - Storage: each weight of the frozen base is snapped to the nearest of 16
+ *    NormalFloat levels and kept in 4 bits, with one absmax scale per block of
+ *    64 weights ("QLoRA: Quantized Low-Rank Adaptation", Piece 1 and the
+ *    section "NF4: a 4-bit format matched to weight statistics"; "QLoRA
+ *    Explained: Fine-Tune 70B+ LLMs on a Single GPU", section "4-Bit
+ *    NormalFloat (NF4) Quantization").
+ *  - Double quantization: the block scales themselves are stored as 8-bit
+ *    floats (OCP E4M3) in blocks of 256 with one fp32 scale per block and one
+ *    fp32 mean offset per tensor ("QLoRA: Quantized Low-Rank Adaptation",
+ *    section "Double quantization (the label-index-card trick)"; "QLoRA
+ *    Explained", section "Double Quantization").
+ *  - Compute: right before the multiply each block is dequantized to BF16
+ *    ("QLoRA: Quantized Low-Rank Adaptation", Piece 2; "Batched 4-bit
+ *    matmuls") and used in
+ *        Y = X W'^T + (alpha/r) (X A^T) B^T ,
+ *    the backward pass computes dX = dY W' + (alpha/r)(dY B) A and the
+ *    adapter gradients dA = (alpha/r)(dY B)^T X, dB = (alpha/r) dY^T (X A^T);
+ *    the quantized base gets no gradient (same page, Piece 3; "What is
+ *    QLoRA?", Key Characteristics: "Backpropagation through quantized
+ *    weights").
+ *
+ * Bit-level format (fixed by this library where the pages are silent):
+ *  - levels L[0..15]: the asymmetric normal-quantile construction with an
+ *    exact zero at L[7] and L[0] = -1, L[15] = +1 (qlora_nf4_levels returns
+ *    them); code(x) = number of fp32 midpoints fp32((L[i]+L[i+1])*0.5) that
+ *    are strictly below x = fp32(w * fp32(1/absmax)); a block whose absmax
+ *    is zero or subnormal is all code 7;
+ *  - packing: byte j of `codes` holds element 2j in bits 0..3 and element
+ *    2j+1 in bits 4..7 (row-major order of W, blocks never reordered);
+ *  - BF16 mode: scale_bf16[b] = bf16_rn(absmax_b);
+ *  - double-quant mode: mean = fp32(S / nblk), S the fp64 sum of all absmax
+ *    values by a pairwise tree over the array zero-padded to a power of two;
+ *    per 256-block j: d = fp32(absmax - mean), dq_scale[j] = fp32(max|d| /
+ *    448) (1 when max|d| = 0), scale_fp8[b] = e4m3_rn_satfinite(fp32(d /
+ *    dq_scale[j]));
+ *  - dequantized weight: bf16_rn(fp32(L[code] * c)) with c = bf16 scale, or
+ *    c = fp32(fp32(e4m3(q) * dq_scale[b/256]) + mean).
+ *
+ * Conventions for every function:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates device memory, never synchronizes, and keeps no state
+ *    between calls other than a read-only level table and a device error word.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Argument errors are detected on the host before anything is enqueued
+ *    and return QLORA_ERR_INVALID / QLORA_ERR_UNSUPPORTED / QLORA_ERR_WORKSPACE;
+ *    a failed launch returns QLORA_ERR_CUDA.
+ *  - Matrices are row-major and contiguous. bf16 tensors are passed as
+ *    uint16_t bit patterns. Every pointer must be 16-byte aligned.
+ *  - Inputs must be finite; non-finite weights give unspecified codes.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qlora_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID = 1,     /* null pointer, bad size, misaligned pointer */
+  QLORA_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels cover */
+  QLORA_ERR_CUDA = 3,        /* a CUDA launch or query failed */
+  QLORA_ERR_WORKSPACE = 4,   /* workspace pointer null or too small */
+  QLORA_ERR_DEVICE = 5       /* a kernel gave up on a bounded wait */
+} qlora_status;
+
+typedef enum {
+  QLORA_SCALE_BF16 = 0,  /* one bf16 absmax per 64 weights */
+  QLORA_SCALE_DQ_FP8 = 1 /* double quantization (bnb_4bit_use_double_quant) */
+} qlora_scale_mode;
+
+typedef enum { QLORA_DTYPE_BF16 = 0, QLORA_DTYPE_FP32 = 1 } qlora_dtype;
+
+enum { QLORA_BLOCKSIZE = 64, QLORA_DQ_BLOCKSIZE = 256 };
+
+/* qlora_linear_bwd flags */
+enum {
+  QLORA_BWD_ACCUMULATE_GRADS = 1, /* dA += ..., dB += ... (gradient accumulation) */
+  QLORA_BWD_ACCUMULATE_DX = 2     /* dX += ... (e.g. two projections reading the same X) */
+};
+
+/*
+ * An NF4 weight W of shape [n, k] (out_features x in_features). Buffers:
+ *   codes       ceil(n*k/2) bytes
+ *   scale_bf16  nblk uint16     (BF16 mode; NULL otherwise)
+ *   scale_fp8   nblk bytes      (double-quant mode)
+ *   dq_scale    nblk2 floats    (double-quant mode)
+ *   dq_mean     1 float         (double-quant mode)
+ * with nblk = ceil(n*k/64), nblk2 = ceil(nblk/256). blocksize must be 64 and
+ * dq_blocksize 256.
+ */
+typedef struct {
+  int64_t n;
+  int64_t k;
+  int32_t blocksize;
+  int32_t dq_blocksize;
+  int32_t mode; /* qlora_scale_mode */
+  int32_t reserved;
+  uint8_t *codes;
+  uint16_t *scale_bf16;
+  uint8_t *scale_fp8;
+  float *dq_scale;
+  float *dq_mean;
+} qlora_nf4_weight;
+
+/* Human-readable name of a status code (static string). */
+const char *qlora_status_string(int status);
+
+/* Library version string. */
+const char *qlora_version(void);
+
+/* Host: writes the 16 fp32 NF4 levels (ascending) the kernels use and the 15
+ * fp32 decision midpoints (mid may be NULL). Always QLORA_OK. */
+int qlora_nf4_levels(float levels[16], float mid[15]);
+
+/* Bytes of device workspace qlora_nf4_quantize needs (0 in BF16 mode). */
+size_t qlora_nf4_quantize_workspace_bytes(int64_t n, int64_t k, int32_t mode);
+
+/*
+ * Quantize W (fp32 [n, k], device) into `w` (buffers and shape set by the
+ * caller). Any n*k >= 1 (the last block may be partial). The double-quant
+ * mode needs `ws` of at least qlora_nf4_quantize_workspace_bytes bytes.
+ * Deterministic: the same input gives the same bytes on every call.
+ */
+int qlora_nf4_quantize(const float *W, qlora_nf4_weight *w, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Dequantize `w` into out_bf16 ([n, k] bf16, device), bit-exact per the format above. */
+int qlora_nf4_dequantize(const qlora_nf4_weight *w, uint16_t *out_bf16, qlora_stream_t stream);
+
+/* Bytes of device workspace qlora_linear_fwd / qlora_linear_bwd need for m
+ * tokens, an [n, k] weight and rank r. */
+size_t qlora_linear_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
+
+/*
+ * Forward: Y[m, n] = X W'^T + (alpha/r) (X A^T) B^T.
+ *   X  [m, k] bf16;  A [r, k] bf16;  B [n, r] bf16;
+ *   Y  [m, n] in y_dtype (qlora_dtype);
+ *   U_save: optional fp32 [m, r] output of U = X A^T (saved for backward).
+ * Requires k % 64 == 0, n % 8 == 0, m >= 1, r in {8, 16, 32, 64, 128}.
+ */
+int qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t m, const uint16_t *A,
+                     const uint16_t *B, int32_t r, float alpha, void *Y, int32_t y_dtype, float *U_save,
+                     void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Backward through the frozen NF4 base:
+ *   dX[m, k] (+)= dY W' + (alpha/r) (dY B) A      (skipped when dX is NULL)
+ *   dA[r, k] (+)= (alpha/r) (dY B)^T X            fp32
+ *   dB[n, r] (+)= (alpha/r) dY^T U, U = X A^T     fp32
+ * U_saved: optional fp32 [m, r] from the forward pass (NULL: recomputed).
+ * flags: QLORA_BWD_ACCUMULATE_GRADS and/or QLORA_BWD_ACCUMULATE_DX.
+ * Same shape rules as qlora_linear_fwd.
+ */
+int qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t m,
+                     const uint16_t *A, const uint16_t *B, int32_t r, float alpha, const float *U_saved,
+                     void *dX, int32_t dx_dtype, float *dA, float *dB, int32_t flags, void *ws,
+                     size_t ws_bytes, qlora_stream_t stream);
+
+/* SiLU-gated MLP glue (bf16 in/out, fp32 math): h = silu(g) * u. */
+int qlora_silu_gate_fwd(const uint16_t *g, const uint16_t *u, uint16_t *h, int64_t count, qlora_stream_t stream);
+
+/* Backward of h = silu(g) * u: dg = dh*u*s*(1 + g*(1-s)), du = dh*g*s, s = sigmoid(g). */
+int qlora_silu_gate_bwd(const uint16_t *dh, const uint16_t *g, const uint16_t *u, uint16_t *dg, uint16_t *du,
+                        int64_t count, qlora_stream_t stream);
+
+/* Number of kernels this library has launched in this process (all calls,
+ * all devices). */
+int64_t qlora_launch_count(void);
+
+/* Device-time measurement of the fused NF4 tensor-core GEMMs (forward Y and
+ * backward dX). Between qlora_timing_begin and qlora_timing_end the library
+ * records a CUDA event pair on the launch stream around each such launch (at
+ * most max_launches; the events are created here, no device memory is
+ * allocated). qlora_timing_end waits for those events and returns the summed
+ * device time in ms, the number of launches timed and their algorithmic
+ * flops, 2 * rows * cols * (reduction + r). Process-wide, not thread-safe. */
+int qlora_timing_begin(int32_t max_launches);
+int qlora_timing_end(double *total_ms, int32_t *launches, double *flops);
+
+/* Reads and clears the device error word (set when a kernel gave up on a
+ * bounded wait). Synchronizes `stream`. Returns QLORA_OK or QLORA_ERR_DEVICE. */
+int qlora_check_device_error(qlora_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */
