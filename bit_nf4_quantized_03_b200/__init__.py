@@ -34,6 +34,7 @@ EXPORTED = (
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_check_device_error",
     "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end",
+    "qlora_nf4_quantize_noalloc",
 )
 
 
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
         "qlora_launch_count": (ctypes.c_int64, []),
         "qlora_timing_begin": (ctypes.c_int, [i32]),
         "qlora_timing_end": (ctypes.c_int, [vp, vp, vp]),
+        "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -236,3 +238,10 @@ def qlora_timing_end():
     _check(lib().qlora_timing_end(ctypes.addressof(ms), ctypes.addressof(n), ctypes.addressof(fl)),
            "qlora_timing_end")
     return ms.value, n.value, fl.value
+
+
+def qlora_nf4_quantize_noalloc(W: torch.Tensor, w: QuantizedWeight, stream=None):
+    """qlora_nf4_quantize for callers that cannot allocate: no workspace, the
+    library's fixed scratch array is used (calls must not overlap on the GPU)."""
+    _check(lib().qlora_nf4_quantize_noalloc(_ptr(W), w.ref(), _stream(stream)), "qlora_nf4_quantize_noalloc")
+    return w

@@ -135,6 +135,27 @@ size_t qlora_nf4_quantize_workspace_bytes(int64_t n, int64_t k, int32_t mode);
  */
 int qlora_nf4_quantize(const float *W, qlora_nf4_weight *w, void *ws, size_t ws_bytes, qlora_stream_t stream);
 
+/*
+ * qlora_nf4_quantize without a workspace: this entry point allocates nothing.
+ * It is for callers that cannot allocate device memory -- a plugin that a
+ * host framework hands only input and output pointers while the framework
+ * owns all device memory, or a latency-critical path that must not call
+ * cudaMalloc (which can synchronize the device). No passage of the pages has
+ * a counterpart; it is an interface convenience of this library.
+ *  - The double-quant scratch is a fixed 16 MiB array inside the library,
+ *    held by every GPU that loads the library until the process exits. It
+ *    covers n*k <= 267,382,784 weights (e.g. 22016 x 8192 needs 11 MiB);
+ *    larger requests return QLORA_ERR_UNSUPPORTED with nothing enqueued.
+ *  - The first call on a device looks up the scratch's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents
+ *    (each call writes every scratch word before reading it). Calls whose
+ *    work overlaps on the GPU -- on different streams, or from different host
+ *    threads -- race on it; serialize them.
+ *  - Results are bit-identical to qlora_nf4_quantize.
+ */
+int qlora_nf4_quantize_noalloc(const float *W, qlora_nf4_weight *w, qlora_stream_t stream);
+
 /* Dequantize `w` into out_bf16 ([n, k] bf16, device), bit-exact per the format above. */
 int qlora_nf4_dequantize(const qlora_nf4_weight *w, uint16_t *out_bf16, qlora_stream_t stream);
 
