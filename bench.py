@@ -373,6 +373,56 @@ def components(dev, peaks) -> dict:
     return out
 
 
+def run_case(args) -> None:
+    """One named launch sequence for profiling (a few launches, no JSON line)."""
+    import torch
+    import bit_nf4_quantized_03_b200 as q
+    from bit_nf4_quantized_03_b200 import build, synth
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name = args.case
+    if name in ("fwd_q_65b", "bwd_q_65b", "fwd_m16_q_65b", "fwd_gate_65b", "bwd_down_65b"):
+        lay = {"fwd_q_65b": LAYERS[0], "bwd_q_65b": LAYERS[0], "fwd_m16_q_65b": LAYERS[0],
+               "fwd_gate_65b": LAYERS[4], "bwd_down_65b": LAYERS[6]}[name]
+        _, n, k = lay
+        m = M_SMALL if name == "fwd_m16_q_65b" else M_TOKENS
+        W = synth.weight(n, k).to(dev)
+        qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+        q.qlora_nf4_quantize(W, qw)
+        del W
+        a, b = (t.to(dev) for t in synth.lora_pair(RANK_R, k, n))
+        x = synth.activations(m, k).to(dev)
+        dy = synth.grad_output(m, n).to(dev)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+        dx = torch.empty(m, k, dtype=torch.bfloat16, device=dev)
+        u = torch.empty(m, RANK_R, dtype=torch.float32, device=dev)
+        da = torch.empty(RANK_R, k, dtype=torch.float32, device=dev)
+        db = torch.empty(n, RANK_R, dtype=torch.float32, device=dev)
+        ws = torch.empty(q.qlora_linear_workspace_bytes(m, n, k, RANK_R), dtype=torch.uint8, device=dev)
+        q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+        for _ in range(args.case_iters):
+            if name.startswith("bwd"):
+                q.qlora_linear_bwd(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, ws)
+            else:
+                q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+    elif name in ("quantize_4096", "dequantize_4096"):
+        W = synth.weight(4096, 4096, outlier_frac=0.001).to(dev)
+        qw = q.QuantizedWeight(4096, 4096, q.QLORA_SCALE_DQ_FP8, device=dev)
+        out = torch.empty(4096, 4096, dtype=torch.bfloat16, device=dev)
+        q.qlora_nf4_quantize(W, qw)
+        for _ in range(args.case_iters):
+            if name == "quantize_4096":
+                q.qlora_nf4_quantize(W, qw)
+            else:
+                q.qlora_nf4_dequantize(qw, out)
+    else:
+        raise SystemExit(f"unknown case {name}")
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    print(f"case {name}: ok, {q.qlora_launch_count()} library launches", flush=True)
+
+
 def run_native(args) -> None:
     import torch
     import torch.distributed as dist
@@ -418,10 +468,13 @@ def run_native(args) -> None:
         wl.h2d()
         wl.step()
         wl.d2h()
-    for _ in range(2):
-        e2e_step()
-    ms_e2e = max_over_ranks(time_steps(e2e_step, args.steps, wl.flush, barrier))
-    e2e_value = flops / (ms_e2e * 1e-3) / 1e12
+    e2e = None
+    if not args.no_e2e:
+        for _ in range(2):
+            e2e_step()
+        ms_e2e = max_over_ranks(time_steps(e2e_step, args.steps, wl.flush, barrier))
+        e2e = {"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": wl.h2d_bytes,
+               "d2h_bytes_per_step": wl.d2h_bytes, "ms_per_step": ms_e2e}
 
     peak_tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
@@ -433,7 +486,7 @@ def run_native(args) -> None:
     comp = None
     cpu = None
     if rank == 0 and world == 1:
-        comp = components(dev, peaks)
+        comp = None if args.no_components else components(dev, peaks)
         if not args.no_cpu_baseline:
             s = OracleSample()
             times = [s.step() for _ in range(args.cpu_steps)]
@@ -452,8 +505,7 @@ def run_native(args) -> None:
                        "parallelism": f"dp{world}", "step_tflop": flops / 1e12 / world},
             "tokens_per_s": tokens_per_s,
             "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": wl.h2d_bytes,
-                    "d2h_bytes_per_step": wl.d2h_bytes, "ms_per_step": ms_e2e},
+            "e2e": e2e,
             "gpu_launches": launches, "clocks": clk.summary(), "components": comp,
         }
         print(json.dumps(line), flush=True)
@@ -469,8 +521,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--cpu-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--case", default=None, help="run one named launch sequence for profiling and exit")
+    ap.add_argument("--case-iters", type=int, default=3)
     args = ap.parse_args(argv)
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_native(args)

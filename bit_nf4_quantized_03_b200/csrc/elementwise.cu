@@ -171,7 +171,33 @@ __global__ void silu_gate_fwd_kernel(const uint16_t* __restrict__ g, const uint1
 __global__ void silu_gate_bwd_kernel(const uint16_t* __restrict__ dh, const uint16_t* __restrict__ g,
                                      const uint16_t* __restrict__ u, uint16_t* __restrict__ dg,
                                      uint16_t* __restrict__ du, int64_t count) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+  const int64_t n8 = count / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 dv = __ldcs(reinterpret_cast<const uint4*>(dh) + i);
+    const uint4 gv = __ldcs(reinterpret_cast<const uint4*>(g) + i);
+    const uint4 uv = __ldcs(reinterpret_cast<const uint4*>(u) + i);
+    const uint32_t da[4] = {dv.x, dv.y, dv.z, dv.w}, ga[4] = {gv.x, gv.y, gv.z, gv.w}, ua[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float d[2] = {__uint_as_float(da[t] << 16), __uint_as_float(da[t] & 0xFFFF0000u)};
+      float gg[2] = {__uint_as_float(ga[t] << 16), __uint_as_float(ga[t] & 0xFFFF0000u)};
+      float uu[2] = {__uint_as_float(ua[t] << 16), __uint_as_float(ua[t] & 0xFFFF0000u)};
+      float rg[2], ru[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float s = sigmoidf_(gg[e]);
+        ru[e] = d[e] * gg[e] * s;
+        rg[e] = d[e] * uu[e] * s * (1.0f + gg[e] * (1.0f - s));
+      }
+      og[t] = pack_bf16x2(rg[0], rg[1]);
+      ou[t] = pack_bf16x2(ru[0], ru[1]);
+    }
+    __stcs(reinterpret_cast<uint4*>(dg) + i, make_uint4(og[0], og[1], og[2], og[3]));
+    __stcs(reinterpret_cast<uint4*>(du) + i, make_uint4(ou[0], ou[1], ou[2], ou[3]));
+  }
+  for (int64_t i = n8 * 8 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float d = bf2f(dh[i]), gg = bf2f(g[i]), uu = bf2f(u[i]);
     const float s = sigmoidf_(gg);
@@ -189,7 +215,7 @@ cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t*
 
 cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,
                                  uint16_t* du, int64_t count, cudaStream_t st) {
-  silu_gate_bwd_kernel<<<blocks_for(count, 256), 256, 0, st>>>(dh, g, u, dg, du, count);
+  silu_gate_bwd_kernel<<<blocks_for((count + 7) / 8, 256), 256, 0, st>>>(dh, g, u, dg, du, count);
   count_launches(1);
   return cudaGetLastError();
 }

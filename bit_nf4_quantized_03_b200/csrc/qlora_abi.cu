@@ -478,6 +478,7 @@ int qlora_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u
   if (count < 0) return QLORA_ERR_INVALID;
   if (count == 0) return QLORA_OK;
   if (dh == nullptr || g == nullptr || u == nullptr || dg == nullptr || du == nullptr) return QLORA_ERR_INVALID;
+  if (!aligned16(dh) || !aligned16(g) || !aligned16(u) || !aligned16(dg) || !aligned16(du)) return QLORA_ERR_INVALID;
   return cuda_status(launch_silu_gate_bwd(dh, g, u, dg, du, count, reinterpret_cast<cudaStream_t>(stream)));
 }
 
