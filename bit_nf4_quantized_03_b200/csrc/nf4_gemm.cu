@@ -413,7 +413,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -422,7 +422,10 @@ bool tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t 
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                        : swizzle == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                        : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -156,7 +156,8 @@ Split choose_split(int64_t tiles, int64_t k_tiles, int sms) {
 struct Plan {
   int r_pad = 64;
   GemmKind down_k = kGemmLoraDownK, down_mn = kGemmLoraDownMN, grad = kGemmLoraGrad;
-  Split u, g, db, da, fwd;
+  Split u, g, db, da, fwd, bwd;
+  int bn = 256;
   size_t off_u32 = 0, off_scaled = 0, off_hi_a = 0, off_lo_a = 0, off_hi_b = 0, off_lo_b = 0, off_part = 0,
          total = 0;
 };
@@ -175,8 +176,12 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   P.g = choose_split(tm, cdiv(n, 64), sms);
   P.db = choose_split(cdiv(n, 128), cdiv(m, 64), sms);
   P.da = choose_split(cdiv(k, 128), cdiv(m, 64), sms);
-  const int64_t fwd_tiles = tm * cdiv(n, 256);
+  P.bn = wgemm_bn(m);
+  const int64_t tok_tiles = cdiv(m, P.bn);
+  const int64_t fwd_tiles = cdiv(n, 128) * tok_tiles;
   if (fwd_tiles * 2 <= sms) P.fwd = choose_split(fwd_tiles, k / 64, sms);
+  const int64_t bwd_tiles = cdiv(k, 128) * tok_tiles;
+  if (bwd_tiles * 2 <= sms) P.bwd = choose_split(bwd_tiles, cdiv(n, 64), sms);
   const size_t rp = static_cast<size_t>(P.r_pad);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -195,7 +200,8 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   part = std::max(part, static_cast<size_t>(P.g.splits) * m * rp);
   part = std::max(part, static_cast<size_t>(P.db.splits) * n * rp);
   part = std::max(part, static_cast<size_t>(P.da.splits) * k * rp);
-  if (P.fwd.splits > 1) part = std::max(part, static_cast<size_t>(P.fwd.splits) * m * cdiv(n, 256) * 256);
+  if (P.fwd.splits > 1) part = std::max(part, static_cast<size_t>(P.fwd.splits) * m * n);
+  if (P.bwd.splits > 1) part = std::max(part, static_cast<size_t>(P.bwd.splits) * m * k);
   P.off_part = take(part * 4);
   P.total = off;
   return P;
@@ -241,7 +247,7 @@ const CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
 // bf16 matrix [rows, cols] row-major, 128-B swizzled boxes of [64 cols, box_rows].
 bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
   return tmap_2d(m, base, kBF16, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
-                 static_cast<uint64_t>(cols) * 2, 64, box_rows, true);
+                 static_cast<uint64_t>(cols) * 2, 64, box_rows, 128);
 }
 
 // Low-rank product U (or G): partial GEMM over the reduction, then finalize.
@@ -258,9 +264,9 @@ int run_lora_down(const Plan& P, bool b_mn, const uint16_t* act, int64_t m, int6
   std::memset(&maps, 0, sizeof(maps));
   bool ok = map_bf16(&maps.a, act, m, red, 128);
   if (!b_mn) {  // adapter A [r, red] is K-major
-    ok = ok && tmap_2d(&maps.b, adapter, kBF16, red, r, red * 2, 64, P.r_pad, true);
+    ok = ok && tmap_2d(&maps.b, adapter, kBF16, red, r, red * 2, 64, P.r_pad, 128);
   } else {      // adapter B [red, r] is MN-major (r contiguous)
-    ok = ok && tmap_2d(&maps.b, adapter, kBF16, r, red, r * 2, 64, 64, true);
+    ok = ok && tmap_2d(&maps.b, adapter, kBF16, r, red, r * 2, 64, 64, 128);
   }
   if (!ok) return QLORA_ERR_CUDA;
   cudaError_t e = launch_gemm(b_mn ? P.down_mn : P.down_k, p, maps, grid_of(p), st);
@@ -281,9 +287,9 @@ int run_lora_grad(const Plan& P, const Split& sp, const uint16_t* act, int64_t m
   p.out_mode = kOutPartial;
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  bool ok = tmap_2d(&maps.a, act, kBF16, rows, m, rows * 2, 64, 64, true);          // [m, rows], MN-major A
-  ok = ok && tmap_2d(&maps.b, hi, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, true);    // [m, r_pad], MN-major B
-  ok = ok && tmap_2d(&maps.b2, lo, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, true);
+  bool ok = tmap_2d(&maps.a, act, kBF16, rows, m, rows * 2, 64, 64, 128);          // [m, rows], MN-major A
+  ok = ok && tmap_2d(&maps.b, hi, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, 128);    // [m, r_pad], MN-major B
+  ok = ok && tmap_2d(&maps.b2, lo, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, 128);
   if (!ok) return QLORA_ERR_CUDA;
   cudaError_t e = launch_gemm(P.grad, p, maps, grid_of(p), st);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
@@ -368,34 +374,34 @@ int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, co
   int rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st);
   if (rc != QLORA_OK) return rc;
 
-  GemmParams p = base_params(m, n, 256, k / 64, P.fwd);
+  // Y^T = W . X^T + B . (sU)^T with W dequantized on the fly (weight as the 128-row operand)
+  GemmParams p = base_params(n, m, P.bn, k / 64, P.fwd);
   p.ext_tiles = P.r_pad / 64;
   p.scales = scale_src(w);
   p.w_kblocks = k / 64;
   p.w_rows = static_cast<int32_t>(n);
+  p.ld_out = n;
   if (P.fwd.splits > 1) {
     p.out = wsb + P.off_part;
-    p.ld_out = static_cast<int64_t>(p.tiles_n) * 256;
-    p.part_stride = m * p.ld_out;
+    p.part_stride = m * n;
     p.out_mode = kOutPartial;
   } else {
     p.out = Y;
-    p.ld_out = n;
     p.out_mode = (y_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
   }
-  GemmMaps maps;
+  WMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  bool ok = map_bf16(&maps.a, X, m, k, 128);
-  ok = ok && tmap_2d(&maps.b, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
-                     static_cast<uint64_t>(k / 2), 32, 256, false);
-  ok = ok && map_bf16(&maps.a2, sU, m, P.r_pad, 128);
-  ok = ok && tmap_2d(&maps.b2, B, kBF16, r, n, r * 2, 64, 256, true);
+  bool ok = map_bf16(&maps.act, X, m, k, static_cast<uint32_t>(P.bn));
+  ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                     static_cast<uint64_t>(k / 2), 32, 128, 32);
+  ok = ok && tmap_2d(&maps.a2, B, kBF16, r, n, r * 2, 64, 128, 128);
+  ok = ok && map_bf16(&maps.b2, sU, m, P.r_pad, static_cast<uint32_t>(P.bn));
   if (!ok) return QLORA_ERR_CUDA;
   const double fwd_flops = 2.0 * double(m) * double(n) * double(k + r);
-  cudaError_t e = launch_gemm(kGemmFwd, p, maps, grid_of(p), st, fwd_flops);
+  cudaError_t e = launch_wgemm(false, P.bn, p, maps, grid_of(p), st, fwd_flops);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   if (P.fwd.splits > 1) {
-    e = launch_splitk_reduce(static_cast<const float*>(p.out), P.fwd.splits, p.part_stride, m, n, p.ld_out, Y,
+    e = launch_splitk_reduce(static_cast<const float*>(p.out), P.fwd.splits, p.part_stride, m, n, n, Y,
                              y_dtype == QLORA_DTYPE_BF16, 0, st);
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
   }
@@ -438,25 +444,37 @@ int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_
   }
 
   if (dX != nullptr) {
-    GemmParams p = base_params(m, k, 256, cdiv(n, 64), Split{});
+    // dX^T = W^T . dY^T + A^T . (sG)^T, W dequantized into the MN-major operand layout
+    GemmParams p = base_params(k, m, P.bn, cdiv(n, 64), P.bwd);
     p.ext_tiles = P.r_pad / 64;
     p.scales = scale_src(w);
     p.w_kblocks = k / 64;
     p.w_rows = static_cast<int32_t>(n);
-    p.out = dX;
     p.ld_out = k;
-    p.out_mode = (dx_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
-    p.accumulate = (flags & QLORA_BWD_ACCUMULATE_DX) ? 1 : 0;
-    GemmMaps maps;
+    const int acc_dx = (flags & QLORA_BWD_ACCUMULATE_DX) ? 1 : 0;
+    if (P.bwd.splits > 1) {
+      p.out = wsb + P.off_part;
+      p.part_stride = m * k;
+      p.out_mode = kOutPartial;
+    } else {
+      p.out = dX;
+      p.out_mode = (dx_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
+      p.accumulate = acc_dx;
+    }
+    WMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    bool ok = map_bf16(&maps.a, dY, m, n, 128);
-    ok = ok && tmap_2d(&maps.b, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
-                       static_cast<uint64_t>(k / 2), 128, 64, false);
-    ok = ok && map_bf16(&maps.a2, sG, m, P.r_pad, 128);
-    ok = ok && tmap_2d(&maps.b2, A, kBF16, k, r, k * 2, 64, 64, true);
+    bool ok = map_bf16(&maps.act, dY, m, n, static_cast<uint32_t>(P.bn));
+    ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                       static_cast<uint64_t>(k / 2), 64, 64, 64);
+    ok = ok && tmap_2d(&maps.a2, A, kBF16, k, r, k * 2, 64, 64, 128);
+    ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(P.bn));
     if (!ok) return QLORA_ERR_CUDA;
     const double dx_flops = 2.0 * double(m) * double(k) * double(n + r);
-    if (launch_gemm(kGemmBwdDx, p, maps, grid_of(p), st, dx_flops) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_wgemm(true, P.bn, p, maps, grid_of(p), st, dx_flops) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (P.bwd.splits > 1 &&
+        launch_splitk_reduce(static_cast<const float*>(p.out), P.bwd.splits, p.part_stride, m, k, k, dX,
+                             dx_dtype == QLORA_DTYPE_BF16, acc_dx, st) != cudaSuccess)
+      return QLORA_ERR_CUDA;
   }
 
   rc = run_lora_grad(P, P.db, dY, m, n, u_hi, u_lo, r, s, dB, 0, acc_grads, wsb, st);

@@ -73,9 +73,9 @@ struct GemmMaps {
   CUtensorMap a, b, a2, b2;    // b = codes for NF4 modes; b2 = lo half for hi/lo mode
 };
 
-// Host helpers (nf4_gemm.cu)
+// Host helpers (nf4_gemm.cu). swizzle: 0 none, 32, 64 or 128 (bytes).
 bool tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle);
 
 // Launch variants
 enum GemmKind : int {
@@ -99,6 +99,21 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps
 void count_launches(int n);
 bool timing_active();
 void timing_record(cudaStream_t st, bool start, double flops);
+
+// ------------------------------------------------------- weight-operand GEMM
+// (nf4_wgemm.cu) D^T[features, tokens] with the dequantized weight as the
+// 128-row MMA operand. GemmParams: rows = features (n forward, k backward),
+// cols = tokens, tiles_m = features / 128, tiles_n = tokens / BN; the output is
+// row-major [tokens, ld_out] (Y or dX), split partials the same way.
+struct WMaps {
+  CUtensorMap act;     // activations [tokens, reduction] bf16, box [64, BN], 128B swizzle
+  CUtensorMap codes;   // packed codes [n, k/2] u8; forward box [32, 128] (32B swizzle), backward [64, 64] (64B)
+  CUtensorMap a2;      // low-rank A-side tile: B_lora [n, r] (forward) or A_lora [r, k] (backward)
+  CUtensorMap b2;      // low-rank B-side tile: s*U or s*G [tokens, r_pad]
+};
+int wgemm_bn(int64_t tokens);
+cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
+                         double algo_flops);
 
 // ------------------------------------------------------------- elementwise
 cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
