@@ -140,6 +140,78 @@ cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_str
 }
 
 // ---------------------------------------------------------------------------
+// U = X A^T for a few tokens on CUDA cores (the tensor-core path would pad the
+// 128-row tile with mostly empty rows). Grid (adapter row j, K slice of 1024):
+// each thread takes 8 consecutive K of its slice for every token, a block
+// reduction gives the slice's partial, and lora_finalize_kernel sums the
+// slices in a fixed order.
+// ---------------------------------------------------------------------------
+constexpr int kSmallSlice = 1024;
+
+template <int MMAX>
+__global__ void __launch_bounds__(128) lora_down_small_kernel(const uint16_t* __restrict__ X, int m, int64_t k,
+                                                              const uint16_t* __restrict__ A, int r_pad,
+                                                              float* __restrict__ part) {
+  __shared__ float red[4][MMAX];
+  const int j = blockIdx.x;
+  const int ks = blockIdx.y;
+  const int64_t kk = static_cast<int64_t>(ks) * kSmallSlice + threadIdx.x * 8;
+  float acc[MMAX];
+#pragma unroll
+  for (int i = 0; i < MMAX; ++i) acc[i] = 0.f;
+  if (kk < k) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * k + kk));
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    float af[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      af[2 * t] = __uint_as_float(aw[t] << 16);
+      af[2 * t + 1] = __uint_as_float(aw[t] & 0xFFFF0000u);
+    }
+#pragma unroll
+    for (int i = 0; i < MMAX; ++i) {
+      if (i < m) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(i) * k + kk));
+        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          acc[i] = fmaf(__uint_as_float(xw[t] << 16), af[2 * t], acc[i]);
+          acc[i] = fmaf(__uint_as_float(xw[t] & 0xFFFF0000u), af[2 * t + 1], acc[i]);
+        }
+      }
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < MMAX; ++i) {
+    float v = acc[i];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) red[warp][i] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < m; i += blockDim.x)
+    part[(static_cast<int64_t>(ks) * m + i) * r_pad + j] = red[0][i] + red[1][i] + red[2][i] + red[3][i];
+}
+
+int lora_down_small_slices(int64_t k) { return static_cast<int>((k + kSmallSlice - 1) / kSmallSlice); }
+
+cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
+                                   int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
+                                   cudaStream_t st) {
+  const int ks = lora_down_small_slices(k);
+  const dim3 grid(static_cast<unsigned>(r), static_cast<unsigned>(ks));
+  if (m <= 16)
+    lora_down_small_kernel<16><<<grid, 128, 0, st>>>(X, static_cast<int>(m), k, A, r_pad, part);
+  else
+    lora_down_small_kernel<64><<<grid, 128, 0, st>>>(X, static_cast<int>(m), k, A, r_pad, part);
+  count_launches(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_lora_finalize(part, ks, m * r_pad, m, r, r_pad, scale, U32, sU, nullptr, nullptr, st);
+}
+
+// ---------------------------------------------------------------------------
 // SiLU-gated glue: h = silu(g) * u ; dg = dh*u*sig*(1 + g*(1-sig)), du = dh*g*sig
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }

@@ -1,22 +1,19 @@
-// Tensor-core GEMM for the frozen-base linear layer and its low-rank branch,
-// sm_100a: TMA-staged operand tiles in 128-byte-swizzled shared memory,
+// Tensor-core GEMM for the low-rank branch of the layer (sm_100a): the
+// skinny products U = X A^T, G = dY B and the adapter gradients dB = dY^T U,
+// dA^T = X^T G. TMA-staged operand tiles in 128-byte-swizzled shared memory,
 // tcgen05.mma (kind::f16, BF16 x BF16 -> FP32) accumulating in TMEM, and a
 // persistent, warp-specialised schedule:
 //
-//   warp 0      TMA producer (activation tiles; packed NF4 codes or bf16 B tiles)
+//   warp 0      TMA producer
 //   warp 1      TMEM allocator + single-thread MMA issuer
 //   warps 2-5   epilogue: TMEM -> registers -> global (one TMEM lane quarter each)
-//   warps 6-13  (NF4 modes) dequantizers: packed 4-bit codes -> BF16 tile in the
-//               exact shared-memory layout the MMA descriptor expects
 //
-// The NF4 weight is never materialised in BF16 in global memory: each 64-weight
-// block is expanded "right before the GPU multiplies" ("QLoRA: Quantized
-// Low-Rank Adaptation", Piece 2; "Batched 4-bit matmuls"). The low-rank
-// branch rides along as extra K steps into the same accumulator:
-//   forward  Y  = [X | s*U] . [W | B]^T            (U = X A^T)
-//   backward dX = [dY | s*G] . [W ; A]              (G = dY B)
-// Accumulators are double-buffered in TMEM so the epilogue of one tile
-// overlaps the main loop of the next.
+// Operands may be K-major or MN-major (the reduction over tokens reads X and
+// dY transposed without a copy); the gradient variant multiplies one A tile
+// by a hi and a lo bf16 B tile into the same accumulator, carrying an fp32
+// operand at ~2^-17 relative precision. The reduction can be split across
+// CTAs into fp32 partials (reduced later in a fixed order). The frozen NF4
+// weight is handled by nf4_wgemm.cu.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -33,18 +30,14 @@ struct GemmCfg {
   static constexpr int BMode = kBMode;
   static constexpr bool Ext = kExt;
   static constexpr bool HiLo = kHiLo;
-  static constexpr bool Nf4 = (kBMode == kB_Nf4K || kBMode == kB_Nf4MN);
-  static constexpr bool BMn = (kBMode == kB_TmaMN || kBMode == kB_Nf4MN);
+  static constexpr bool BMn = (kBMode == kB_TmaMN);
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBTile = BN * 64 * 2;
   static constexpr int kBBytes = kBTile * (HiLo ? 2 : 1);
-  static constexpr int kRBytes = Nf4 ? BN * 32 : 0;
-  static constexpr int kDeqWarps = Nf4 ? 8 : 0;
-  static constexpr int kThreads = (6 + kDeqWarps) * 32;
+  static constexpr int kThreads = 6 * 32;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = Stages * (kABytes + kBBytes + kRBytes) + 1024 + kBarBytes;
-  static_assert(!Nf4 || BN == 256, "dequantizer thread mapping assumes a 256-wide tile");
+  static constexpr int kSmemBytes = Stages * (kABytes + kBBytes) + 1024 + kBarBytes;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM alloc size");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -152,12 +145,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::Stages * C::kABytes;
-  uint8_t* sR = sB + C::Stages * C::kBBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + C::Stages * C::kRBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::Stages * C::kBBytes);
   uint64_t* tma_full = bars;
-  uint64_t* deq_full = bars + C::Stages;
-  uint64_t* empty = bars + 2 * C::Stages;
-  uint64_t* acc_full = bars + 3 * C::Stages;
+  uint64_t* empty = bars + C::Stages;
+  uint64_t* acc_full = bars + 2 * C::Stages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
@@ -168,7 +159,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::Stages; ++s) {
       mbar_init(&tma_full[s], 1);
-      mbar_init(&deq_full[s], C::kDeqWarps > 0 ? C::kDeqWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -209,7 +199,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           uint64_t* bar = &tma_full[stage];
           if (i < nmain) {
             const int kt = kt0 + i;
-            mbar_arrive_expect_tx(bar, C::kABytes + (C::Nf4 ? C::kRBytes : C::kBBytes));
+            mbar_arrive_expect_tx(bar, C::kABytes + C::kBBytes);
             if (C::AMn) {
               tma_load_2d(a_dst, &maps.a, bar, mb * 128, kt * 64);
               tma_load_2d(a_dst + 8192, &maps.a, bar, mb * 128 + 64, kt * 64);
@@ -218,16 +208,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             }
             if (C::BMode == kB_TmaK) {
               tma_load_2d(b_dst, &maps.b, bar, kt * 64, nb * C::BN);
-            } else if (C::BMode == kB_TmaMN) {
+            } else {
 #pragma unroll
               for (int j = 0; j < C::BN / 64; ++j) {
                 tma_load_2d(b_dst + j * 8192, &maps.b, bar, nb * C::BN + 64 * j, kt * 64);
                 if (C::HiLo) tma_load_2d(b_dst + C::kBTile + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, kt * 64);
               }
-            } else if (C::BMode == kB_Nf4K) {
-              tma_load_2d(sR + stage * C::kRBytes, &maps.b, bar, kt * 32, nb * C::BN);
-            } else {
-              tma_load_2d(sR + stage * C::kRBytes, &maps.b, bar, nb * (C::BN / 2), kt * 64);
             }
           } else {
             const int e = i - nmain;
@@ -276,7 +262,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int i = 0; i < nmain + next; ++i) {
           if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
-          if (C::Nf4 && !mbar_wait(&deq_full[stage], ph)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
           const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
@@ -326,65 +311,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       acc ^= 1;
       if (acc == 0) aph ^= 1;
-    }
-  } else if (C::Nf4) {
-    // ------------------------------------------------------------ dequantizers
-    const int dt = threadIdx.x - 192;           // 0..255
-    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
-    // K-major (forward): thread = W row inside the 256-row tile.
-    // MN-major (backward): thread = (W row i of the 64-row K step, 64-col chunk c).
-    const int i_mn = dt & 63;
-    const int c_mn = dt >> 6;
-    const int srow = (C::BMode == kB_Nf4K) ? dt : i_mn;     // row whose 128-B line we write
-    const int sw = srow & 7;
-    const uint32_t r_off = (C::BMode == kB_Nf4K) ? static_cast<uint32_t>(dt * 32)
-                                                 : static_cast<uint32_t>(i_mn * (C::BN / 2) + c_mn * 32);
-    const uint32_t b_off = (C::BMode == kB_Nf4K)
-                               ? static_cast<uint32_t>((dt >> 3) * 1024 + (dt & 7) * 128)
-                               : static_cast<uint32_t>(c_mn * 8192 + (i_mn >> 3) * 1024 + (i_mn & 7) * 128);
-    int stage = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-      int mb, nb, split, kt0, nmain, next;
-      decode_unit(p, u, mb, nb, split, kt0, nmain, next);
-      for (int i = 0; i < nmain + next; ++i) {
-        if (i < nmain) {
-          const int kt = kt0 + i;
-          int64_t wrow, kb;
-          if (C::BMode == kB_Nf4K) { wrow = static_cast<int64_t>(nb) * C::BN + dt; kb = kt; }
-          else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(nb) * (C::BN / 64) + c_mn; }
-          const bool valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
-          const float c = valid ? block_scale(p.scales, wrow * p.w_kblocks + kb, mean) : 0.f;
-          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
-          const uint32_t bdst = smem_u32(sB + stage * C::kBBytes) + b_off;
-          if (valid) {
-            const uint32_t rsrc = smem_u32(sR + stage * C::kRBytes) + r_off;
-            const uint4 w0 = ld_shared_v4(rsrc);
-            const uint4 w1 = ld_shared_v4(rsrc + 16);
-            const Nf4Lut lut = nf4_build_lut(p.tab, c);
-            st_shared_v4(bdst + ((0 ^ sw) << 4), nf4_lookup8(lut, w0.x));
-            st_shared_v4(bdst + ((1 ^ sw) << 4), nf4_lookup8(lut, w0.y));
-            st_shared_v4(bdst + ((2 ^ sw) << 4), nf4_lookup8(lut, w0.z));
-            st_shared_v4(bdst + ((3 ^ sw) << 4), nf4_lookup8(lut, w0.w));
-            st_shared_v4(bdst + ((4 ^ sw) << 4), nf4_lookup8(lut, w1.x));
-            st_shared_v4(bdst + ((5 ^ sw) << 4), nf4_lookup8(lut, w1.y));
-            st_shared_v4(bdst + ((6 ^ sw) << 4), nf4_lookup8(lut, w1.z));
-            st_shared_v4(bdst + ((7 ^ sw) << 4), nf4_lookup8(lut, w1.w));
-          } else {
-            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) st_shared_v4(bdst + (j << 4), z);
-          }
-          fence_proxy_async_smem();
-        } else {
-          // extension step: the producer loads the tile; only keep the phases in step
-          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&deq_full[stage]);
-        if (++stage == C::Stages) { stage = 0; ph ^= 1; }
-      }
     }
   }
 
@@ -450,8 +376,6 @@ static cudaError_t launch_cfg(const GemmParams& p, const GemmMaps& maps, int gri
   return cudaGetLastError();
 }
 
-using CfgFwd = GemmCfg<256, 4, false, kB_Nf4K, true, false>;
-using CfgBwd = GemmCfg<256, 4, false, kB_Nf4MN, true, false>;
 using CfgDownK = GemmCfg<64, 6, false, kB_TmaK, false, false>;
 using CfgDownMN = GemmCfg<64, 6, false, kB_TmaMN, false, false>;
 using CfgGrad = GemmCfg<64, 6, true, kB_TmaMN, false, true>;
@@ -461,7 +385,6 @@ using CfgGrad128 = GemmCfg<128, 4, true, kB_TmaMN, false, true>;
 
 int gemm_bn(GemmKind kind) {
   switch (kind) {
-    case kGemmFwd: case kGemmBwdDx: return 256;
     case kGemmLoraDownK128: case kGemmLoraDownMN128: case kGemmLoraGrad128: return 128;
     default: return 64;
   }
@@ -470,8 +393,6 @@ int gemm_bn(GemmKind kind) {
 static cudaError_t launch_gemm_impl(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid,
                                     cudaStream_t st) {
   switch (kind) {
-    case kGemmFwd: return launch_cfg<CfgFwd>(p, maps, grid, st);
-    case kGemmBwdDx: return launch_cfg<CfgBwd>(p, maps, grid, st);
     case kGemmLoraDownK: return launch_cfg<CfgDownK>(p, maps, grid, st);
     case kGemmLoraDownMN: return launch_cfg<CfgDownMN>(p, maps, grid, st);
     case kGemmLoraGrad: return launch_cfg<CfgGrad>(p, maps, grid, st);
@@ -482,12 +403,8 @@ static cudaError_t launch_gemm_impl(GemmKind kind, const GemmParams& p, const Ge
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st,
-                        double algo_flops) {
-  const bool timed = (kind == kGemmFwd || kind == kGemmBwdDx) && timing_active();
-  if (timed) timing_record(st, true, algo_flops);
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st) {
   const cudaError_t e = launch_gemm_impl(kind, p, maps, grid, st);
-  if (timed) timing_record(st, false, algo_flops);
   count_launches(1);
   return e;
 }

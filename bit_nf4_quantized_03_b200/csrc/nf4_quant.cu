@@ -18,81 +18,157 @@ __device__ int g_device_error = 0;
 
 // ---------------------------------------------------------------------------
 // Stage 1: absmax, codes, plain scales / fp32 absmax for double quant.
-// Each half-warp owns one 64-block: 16 lanes x float4 (128-bit loads).
+//
+// The weights stream through a 3-stage shared-memory ring filled by bulk
+// copies (32 KB chunks of 128 blocks). Eight lanes share one 64-block (eight
+// weights each, two conflict-free 128-bit shared reads), so the per-block
+// work -- absmax over the eight lanes, the IEEE reciprocal, the scale store --
+// is spread over eight weights per lane.
+//
+// The code of x = w * (1/absmax) is found with one comparison: [-1 - 1/16,
+// 1 + 1/16) is cut into 35 buckets of width 1/16, each widened by 1e-3; the
+// widened bucket holds at most one decision threshold (neighbouring
+// thresholds are >= 0.08 apart), so code = (thresholds below the bucket) +
+// (x > the bucket's threshold), exactly the number of thresholds strictly
+// below x. The bucket index only has to be right up to the widening, which
+// covers the rounding of x * 16 + 16.5 and of the round-to-integer below.
+//
+// In double-quant mode each chunk's 128 absmax values are also reduced in
+// fp64 with the fixed pairwise tree (the first levels of the tensor-wide sum
+// that defines the mean).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Table& t) {
-  // number of thresholds strictly below x (a value on a threshold rounds down)
-  uint32_t c = 0;
-#pragma unroll
-  for (int i = 0; i < 15; ++i) c += (x > t.mid[i]) ? 1u : 0u;
-  return c;
+constexpr int kQChunk = 128;     // 64-blocks per chunk: 32 KB of fp32 weights
+constexpr int kQStages = 3;
+constexpr int kQSmem = kQStages * kQChunk * 256;
+
+__device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2* tab) {
+  // bucket = floor(x * 16 + 17): round-to-integer of x * 16 + 16.5 by adding 1.5 * 2^23
+  const float r = __fadd_rn(__fmaf_rn(x, 16.0f, 16.5f), 12582912.0f);
+  const float2 e = tab[__float_as_uint(r) & 63u];
+  return static_cast<uint32_t>(__float_as_int(e.y)) + ((x > e.x) ? 1u : 0u);
 }
 
 template <bool kDQ>
-__global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restrict__ W, int64_t n_elem,
-                                                           Nf4Table tab, uint8_t* __restrict__ codes,
-                                                           uint16_t* __restrict__ scale_bf16,
-                                                           float* __restrict__ absmax_out) {
-  const int lane = threadIdx.x & 31;
-  const int hl = lane & 15;
-  const int64_t nfull = n_elem / 64;                     // complete blocks
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const float4* W4 = reinterpret_cast<const float4*>(W);
-
-  constexpr int U = 4;   // block pairs in flight per warp
-  for (int64_t base = warp * 2 * U; base < nfull; base += nwarps * 2 * U) {
-    float4 v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t b = base + 2 * u + (lane >> 4);
-      v[u] = (b < nfull) ? __ldcs(W4 + b * 16 + hl) : make_float4(0.f, 0.f, 0.f, 0.f);
+__global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __restrict__ W, int64_t n_elem,
+                                                              Nf4Buckets bk, uint8_t* __restrict__ codes,
+                                                              uint16_t* __restrict__ scale_bf16,
+                                                              float* __restrict__ absmax_out,
+                                                              double* __restrict__ part_out) {
+  extern __shared__ __align__(128) uint8_t q_stage[];
+  __shared__ float2 s_tab[64];
+  __shared__ double s_tree[kQChunk];
+  __shared__ __align__(8) uint64_t full[kQStages];
+  const int tid = threadIdx.x;
+  const int grp = tid >> 3;          // one 64-block per group of eight lanes
+  const int l = tid & 7;
+  const int64_t nfull = n_elem / 64;
+  const int64_t tail = n_elem - nfull * 64;
+  const int64_t nblk = nfull + (tail > 0 ? 1 : 0);
+  const int64_t nchunks = (nblk + kQChunk - 1) / kQChunk;
+  const int64_t my_n = (nchunks > blockIdx.x) ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (tid < 64) {
+    // entry b covers [(b - 1)/16 - 1, b/16 - 1); entries 0 and 34 are the padding buckets
+    const int b = tid;
+    s_tab[b] = (b < 35) ? make_float2(bk.thr[b], __int_as_float(bk.base[b]))
+                        : make_float2(__int_as_float(0x7f800000), __int_as_float(15));
+  }
+  if (tid == 0) {
+    for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t i) {
+    const int64_t b0 = (blockIdx.x + i * gridDim.x) * kQChunk;
+    int64_t nb = nfull - b0;
+    nb = nb < 0 ? 0 : (nb > kQChunk ? kQChunk : nb);
+    const int st = static_cast<int>(i % kQStages);
+    if (nb > 0) {
+      mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nb * 256));
+      bulk_load(q_stage + st * (kQChunk * 256), W + b0 * 64, static_cast<uint32_t>(nb * 256), &full[st]);
+    } else {
+      mbar_arrive(&full[st]);
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t b = base + 2 * u + (lane >> 4);
-      float m = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      uint32_t q;
-      if (m < 1.17549435e-38f) {          // zero or subnormal absmax: exact-zero level
-        q = 0x7777u;
-      } else {
-        const float inv = __frcp_rn(m);
-        q = nf4_code(__fmul_rn(v[u].x, inv), tab) | (nf4_code(__fmul_rn(v[u].y, inv), tab) << 4) |
-            (nf4_code(__fmul_rn(v[u].z, inv), tab) << 8) | (nf4_code(__fmul_rn(v[u].w, inv), tab) << 12);
-      }
+  };
+  if (tid == 0)
+    for (int64_t i = 0; i < my_n && i < kQStages; ++i) issue(i);
+  const uint32_t x = (l >> 2) & 1;   // which half of its 32 bytes a lane reads first (bank-conflict free)
+  for (int64_t i = 0; i < my_n; ++i) {
+    const int st = static_cast<int>(i % kQStages);
+    if (!mbar_wait(&full[st], static_cast<uint32_t>((i / kQStages) & 1))) break;
+    const int64_t b0 = (blockIdx.x + i * gridDim.x) * kQChunk;
+    const uint32_t sbase = smem_u32(q_stage + st * (kQChunk * 256));
+#pragma unroll 2
+    for (int it = 0; it < kQChunk / 32; ++it) {
+      const int lb = it * 32 + grp;
+      const int64_t b = b0 + lb;
+      float v[8];
       if (b < nfull) {
-        reinterpret_cast<uint16_t*>(codes)[b * 16 + hl] = static_cast<uint16_t>(q);
-        if (hl == 0) {
-          if (kDQ) absmax_out[b] = m;
-          else scale_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
+        const uint32_t src = sbase + lb * 256 + l * 32;
+        float4 h0, h1;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(h0.x), "=f"(h0.y), "=f"(h0.z), "=f"(h0.w) : "r"(src + 16 * x) : "memory");
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(h1.x), "=f"(h1.y), "=f"(h1.z), "=f"(h1.w) : "r"(src + 16 * (x ^ 1)) : "memory");
+        const float4 lo = x ? h1 : h0;
+        const float4 hi = x ? h0 : h1;
+        v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+        v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int64_t idx = 8 * l + e;
+          v[e] = (b == nfull && idx < tail) ? W[b * 64 + idx] : 0.f;
         }
       }
-    }
-  }
-
-  // ragged last block (n_elem % 64 != 0): one warp, scalar loads
-  const int64_t tail = n_elem - nfull * 64;
-  if (tail > 0 && blockIdx.x == 0 && threadIdx.x < 32) {
-    const int64_t b = nfull;
-    float w0 = (2 * lane < tail) ? W[b * 64 + 2 * lane] : 0.f;
-    float w1 = (2 * lane + 1 < tail) ? W[b * 64 + 2 * lane + 1] : 0.f;
-    float m = fmaxf(fabsf(w0), fabsf(w1));
+      float m = fabsf(v[0]);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    uint32_t c0 = 7, c1 = 7;
-    if (m >= 1.17549435e-38f) {
-      const float inv = __frcp_rn(m);
-      c0 = nf4_code(__fmul_rn(w0, inv), tab);
-      c1 = nf4_code(__fmul_rn(w1, inv), tab);
+      for (int e = 1; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      uint32_t word = 0x77777777u;      // zero or subnormal absmax: the exact-zero level
+      if (m >= 1.17549435e-38f) {
+        const float inv = __frcp_rn(m);
+        word = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) word |= nf4_code_bucket(__fmul_rn(v[e], inv), s_tab) << (4 * e);
+      }
+      if (b < nfull) {
+        reinterpret_cast<uint32_t*>(codes)[b * 8 + l] = word;
+      } else if (b == nfull && tail > 0) {
+        // ragged last block: only the bytes that hold present elements; an odd tail keeps its high nibble 0
+#pragma unroll
+        for (int byte = 0; byte < 4; ++byte) {
+          const int64_t e0 = 8 * l + 2 * byte;
+          if (e0 < tail) {
+            uint32_t c = (word >> (8 * byte)) & 0xFFu;
+            if (e0 + 1 >= tail) c &= 0x0Fu;
+            codes[b * 32 + 4 * l + byte] = static_cast<uint8_t>(c);
+          }
+        }
+      }
+      if (l == 0 && b < nblk) {
+        if (kDQ) absmax_out[b] = m;
+        else scale_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
+      }
+      if (kDQ && l == 0) s_tree[lb] = (b < nblk) ? static_cast<double>(m) : 0.0;
     }
-    if (2 * lane + 1 >= tail) c1 = 0;    // odd tail: high nibble stays 0
-    if (2 * lane < tail) codes[b * 32 + lane] = static_cast<uint8_t>(c0 | (c1 << 4));
-    if (lane == 0) {
-      if (kDQ) absmax_out[b] = m;
-      else scale_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
+    __syncthreads();                          // stage consumed, tree leaves written
+    if (kDQ) {
+      // fixed pairwise tree over this chunk's 128 absmax values
+      double t = 0.0;
+      if (tid < kQChunk / 2) t = s_tree[2 * tid] + s_tree[2 * tid + 1];
+      __syncthreads();
+      if (tid < kQChunk / 2) s_tree[tid] = t;
+      __syncthreads();
+      for (int stride = 1; stride < kQChunk / 2; stride <<= 1) {
+        if (tid < kQChunk / 2 && (tid & (2 * stride - 1)) == 0) s_tree[tid] = s_tree[tid] + s_tree[tid + stride];
+        __syncthreads();
+      }
+      if (tid == 0) part_out[blockIdx.x + i * gridDim.x] = s_tree[0];
+      __syncthreads();
     }
+    if (tid == 0 && i + kQStages < my_n) issue(i + kQStages);
   }
 }
 
@@ -155,97 +231,171 @@ __global__ void __launch_bounds__(256) dq_fp8_kernel(const float* __restrict__ a
 }
 
 // ---------------------------------------------------------------------------
-// Standalone dequantization: one thread per 64-block, table lookups, 128-bit
-// loads of codes and 128-bit stores of bf16.
+// Standalone dequantization. The codes of 256 consecutive blocks (one
+// second-level scale block, 8 KB) are streamed into a 3-stage shared-memory
+// ring by bulk copies; each lane expands one 64-block through the per-block
+// lookup table into a 128-byte row of a per-warp stage (16-byte chunks
+// XOR-swizzled by the row, conflict-free), and the warp then writes its 32
+// rows (4 KB of contiguous output) with fully coalesced 512-byte stores.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __restrict__ codes, ScaleSrc ss,
-                                                             int64_t n_elem, Nf4Table tab,
-                                                             uint16_t* __restrict__ out) {
+constexpr int kDChunk = 256;
+constexpr int kDStages = 3;
+constexpr int kDSmem = kDStages * kDChunk * 32 + 8 * 4096;
+
+__global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* __restrict__ codes, ScaleSrc ss,
+                                                                int64_t n_elem, Nf4Table tab,
+                                                                uint16_t* __restrict__ out) {
+  extern __shared__ __align__(128) uint8_t d_smem[];
+  __shared__ __align__(8) uint64_t full[kDStages];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int64_t nfull = n_elem / 64;
+  const int64_t nchunks = (nfull + kDChunk - 1) / kDChunk;
+  const int64_t my_n = (nchunks > blockIdx.x) ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const float mean = (ss.dq_mean != nullptr) ? __ldg(ss.dq_mean) : 0.f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nfull; b += stride) {
-    const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
-    const uint4 c0 = __ldcs(src);
-    const uint4 c1 = __ldcs(src + 1);
-    const Nf4Lut lut = nf4_build_lut(tab, block_scale(ss, b, mean));
-    uint4* dst = reinterpret_cast<uint4*>(out + b * 64);
-    __stcs(dst + 0, nf4_lookup8(lut, c0.x));
-    __stcs(dst + 1, nf4_lookup8(lut, c0.y));
-    __stcs(dst + 2, nf4_lookup8(lut, c0.z));
-    __stcs(dst + 3, nf4_lookup8(lut, c0.w));
-    __stcs(dst + 4, nf4_lookup8(lut, c1.x));
-    __stcs(dst + 5, nf4_lookup8(lut, c1.y));
-    __stcs(dst + 6, nf4_lookup8(lut, c1.z));
-    __stcs(dst + 7, nf4_lookup8(lut, c1.w));
+  uint8_t* ring = d_smem;
+  const uint32_t stage_out = smem_u32(d_smem + kDStages * kDChunk * 32 + warp * 4096);
+  if (tid == 0) {
+    for (int st = 0; st < kDStages; ++st) mbar_init(&full[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int64_t i) {
+    const int64_t b0 = (blockIdx.x + i * gridDim.x) * kDChunk;
+    int64_t nb = nfull - b0;
+    nb = nb > kDChunk ? kDChunk : nb;
+    const int st = static_cast<int>(i % kDStages);
+    mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nb * 32));
+    bulk_load(ring + st * (kDChunk * 32), codes + b0 * 32, static_cast<uint32_t>(nb * 32), &full[st]);
+  };
+  if (tid == 0)
+    for (int64_t i = 0; i < my_n && i < kDStages; ++i) issue(i);
+  const uint32_t x = (lane >> 2) & 1;           // read order that keeps the two 16-byte loads conflict-free
+  for (int64_t i = 0; i < my_n; ++i) {
+    const int st = static_cast<int>(i % kDStages);
+    const int64_t b0 = (blockIdx.x + i * gridDim.x) * kDChunk + warp * 32;
+    const int64_t b = b0 + lane;
+    // scale loads go out before the wait so their latency overlaps it
+    float c = 0.f;
+    if (b < nfull) c = block_scale(ss, b, mean);
+    if (!mbar_wait(&full[st], static_cast<uint32_t>((i / kDStages) & 1))) break;
+    if (b < nfull) {
+      const uint32_t src = smem_u32(ring + st * (kDChunk * 32) + (warp * 32 + lane) * 32);
+      uint4 h0, h1;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(h0.x), "=r"(h0.y), "=r"(h0.z), "=r"(h0.w) : "r"(src + 16 * x) : "memory");
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(h1.x), "=r"(h1.y), "=r"(h1.z), "=r"(h1.w) : "r"(src + 16 * (x ^ 1)) : "memory");
+      const uint4 c0 = x ? h1 : h0;
+      const uint4 c1 = x ? h0 : h1;
+      const Nf4Lut lut = nf4_build_lut(tab, c);
+      const uint32_t row = stage_out + lane * 128;
+      const int sw = lane & 7;
+      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 v = nf4_lookup8(lut, words[j]);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((j ^ sw) << 4)), "r"(v.x), "r"(v.y),
+                     "r"(v.z), "r"(v.w)
+                     : "memory");
+      }
+    }
+    __syncwarp();
+    const int64_t nvalid = (nfull - b0 < 32) ? (nfull - b0) : 32;
+    uint4* dst = reinterpret_cast<uint4*>(out + b0 * 64);
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int o = it * 512 + lane * 16;     // byte offset in the warp's 4 KB of output
+      const int blk = o >> 7;
+      const int chunk = (o >> 4) & 7;
+      if (blk < nvalid) {
+        uint4 v;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(stage_out + blk * 128 + ((chunk ^ (blk & 7)) << 4))
+                     : "memory");
+        __stcs(dst + (o >> 4), v);
+      }
+    }
+    __syncthreads();                           // code stage consumed by every warp
+    if (tid == 0 && i + kDStages < my_n) issue(i + kDStages);
   }
   const int64_t tail = n_elem - nfull * 64;
-  if (tail > 0 && blockIdx.x == 0 && threadIdx.x < tail) {
+  if (tail > 0 && blockIdx.x == 0 && tid < tail) {
     const int64_t b = nfull;
-    const int i = threadIdx.x;
-    const uint8_t byte = codes[b * 32 + i / 2];
-    const uint32_t code = (i & 1) ? (byte >> 4) : (byte & 15u);
+    const int e = tid;
+    const uint8_t byte = codes[b * 32 + e / 2];
+    const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 15u);
     const Nf4Lut lut = nf4_build_lut(tab, block_scale(ss, b, mean));
     uint32_t v01, v23;
     nf4_lookup4(lut, code, v01, v23);
-    out[b * 64 + i] = static_cast<uint16_t>(v01 & 0xFFFFu);
+    out[b * 64 + e] = static_cast<uint16_t>(v01 & 0xFFFFu);
   }
 }
 
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-static int grid_for(int64_t work_items, int per_cta, int max_ctas) {
-  int64_t g = (work_items + per_cta - 1) / per_cta;
-  if (g < 1) g = 1;
-  if (g > max_ctas) g = max_ctas;
-  return static_cast<int>(g);
+
+template <typename K>
+static cudaError_t set_smem_once(K kernel, int bytes, bool* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
 }
 
-cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab, uint8_t* codes,
-                            uint16_t* scale_bf16, uint8_t* scale_fp8, float* dq_scale, float* dq_mean,
-                            void* ws, int num_sms, cudaStream_t st) {
+cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab, const Nf4Buckets& bk,
+                            uint8_t* codes, uint16_t* scale_bf16, uint8_t* scale_fp8, float* dq_scale,
+                            float* dq_mean, void* ws, int num_sms, cudaStream_t st) {
+  (void)tab;
+  static bool smem_set[2][64] = {};
   const int64_t nblk = (n_elem + 63) / 64;
   const bool dq = (scale_fp8 != nullptr);
-  // each warp covers 8 blocks per iteration; aim for several waves of 8 warps per SM
-  const int grid = grid_for((nblk + 63) / 64, 1, num_sms * 8);
-  float* absmax = reinterpret_cast<float*>(ws);
-  if (dq) {
-    nf4_quantize_kernel<true><<<grid, 256, 0, st>>>(W, n_elem, tab, codes, nullptr, absmax);
-    count_launches(1);
-  } else {
-    nf4_quantize_kernel<false><<<grid, 256, 0, st>>>(W, n_elem, tab, codes, scale_bf16, nullptr);
+  const int64_t nchunks = (nblk + kQChunk - 1) / kQChunk;
+  const int grid = static_cast<int>(nchunks < 2LL * num_sms ? nchunks : 2LL * num_sms);
+  cudaError_t e;
+  if (!dq) {
+    e = set_smem_once(nf4_quantize_kernel<false>, kQSmem, smem_set[0]);
+    if (e != cudaSuccess) return e;
+    nf4_quantize_kernel<false><<<grid, 256, kQSmem, st>>>(W, n_elem, bk, codes, scale_bf16, nullptr, nullptr);
     count_launches(1);
     return cudaGetLastError();
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // fixed-order fp64 sum -> mean (into the ws slot after the partial sums)
   const QuantWsLayout L = quant_ws_layout(n_elem);
+  float* absmax = reinterpret_cast<float*>(static_cast<char*>(ws) + L.absmax_off);
   double* part_a = reinterpret_cast<double*>(static_cast<char*>(ws) + L.part_a_off);
   double* part_b = reinterpret_cast<double*>(static_cast<char*>(ws) + L.part_b_off);
   float* mean_tmp = reinterpret_cast<float*>(static_cast<char*>(ws) + L.mean_off);
-  int64_t n = nblk;
-  int64_t g = (n + 511) / 512;
-  pairwise_sum_pass<float><<<static_cast<int>(g), 256, 0, st>>>(absmax, n, part_a, nblk,
-                                                                 g == 1 ? mean_tmp : nullptr);
+  // stage 1 also writes one fp64 tree sum per 128 blocks (the first levels of the fixed-order sum)
+  e = set_smem_once(nf4_quantize_kernel<true>, kQSmem, smem_set[1]);
+  if (e != cudaSuccess) return e;
+  nf4_quantize_kernel<true><<<grid, 256, kQSmem, st>>>(W, n_elem, bk, codes, nullptr, absmax, part_a);
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // remaining levels: aligned chunks of 512 -> 1 until one value is left, then the mean
   double* src = part_a;
   double* dst = part_b;
-  while (g > 1) {
-    n = g;
-    g = (n + 511) / 512;
-    pairwise_sum_pass<double><<<static_cast<int>(g), 256, 0, st>>>(src, n, dst, nblk,
-                                                                    g == 1 ? mean_tmp : nullptr);
+  int64_t n = nchunks;
+  do {
+    const int64_t g = (n + 511) / 512;
+    pairwise_sum_pass<double><<<static_cast<int>(g), 256, 0, st>>>(src, n, dst, nblk, g == 1 ? mean_tmp : nullptr);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     double* t = src;
     src = dst;
     dst = t;
-  }
+    n = g;
+  } while (n > 1);
   const int64_t nb2 = (nblk + 255) / 256;
   dq_fp8_kernel<<<static_cast<int>(nb2), 256, 0, st>>>(absmax, nblk, mean_tmp, scale_fp8, dq_scale, dq_mean);
   count_launches(1);
@@ -254,9 +404,14 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
 
 cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t n_elem, const Nf4Table& tab,
                               uint16_t* out, int num_sms, cudaStream_t st) {
-  const int64_t nblk = (n_elem + 63) / 64;
-  const int grid = grid_for(nblk, 256, num_sms * 8);
-  nf4_dequantize_kernel<<<grid, 256, 0, st>>>(codes, ss, n_elem, tab, out);
+  static bool smem_set[64] = {};
+  const cudaError_t e = set_smem_once(nf4_dequantize_kernel, kDSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  const int64_t nfull = n_elem / 64;
+  const int64_t nchunks = (nfull + kDChunk - 1) / kDChunk;
+  int64_t grid = nchunks < 3LL * num_sms ? nchunks : 3LL * num_sms;
+  if (grid < 1) grid = 1;
+  nf4_dequantize_kernel<<<static_cast<int>(grid), 256, kDSmem, st>>>(codes, ss, n_elem, tab, out);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -7,17 +7,19 @@
 // GPU multiplies", "QLoRA: Quantized Low-Rank Adaptation", Piece 2 and
 // "Batched 4-bit matmuls") straight into the 128-byte-swizzled shared-memory
 // tile that the tcgen05.mma descriptor reads, and is then reused by every
-// token of the tile (up to 256: the MMA's N). Putting W on the 128-row side
-// halves the dequantization per flop compared with a 128-token tile, and at a
-// handful of tokens (M = 16) it wastes no tensor-core rows on padding.
+// token of the tile: one MMA covers up to 256 tokens (its N), and for long
+// token counts two MMAs (two TMEM accumulators of 192 columns) share the same
+// weight tile, so each dequantized weight serves 384 tokens. Putting W on the
+// 128-row side is what makes this reuse possible, and at a handful of tokens
+// (M = 16) it wastes no tensor-core rows on padding.
 //
 // Warp roles (448 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA: packed codes (32B/64B-swizzled so the reads below are
 //               bank-conflict free), activation tiles, low-rank extension tiles
 //   warp 1      TMEM allocation + single-thread tcgen05.mma issue
 //   warps 2-5   epilogue: TMEM -> registers -> global (row-major Y / dX)
-//   warps 6-13  dequantizers in two groups of four; group g owns the stages
-//               with index parity g, so two K steps are expanded concurrently
+//   warps 6-13  dequantizers: two lanes per weight row (32 codes each) expand
+//               every K step of the 128-row tile
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -26,20 +28,31 @@
 
 namespace qlora {
 
-template <int kBN, int kStages, bool kBwd>
+template <int kBN, int kNAcc, int kStages, bool kBwd, int kGroups = 2>
 struct WCfg {
-  static constexpr int BN = kBN;            // tokens per tile (MMA N)
-  static constexpr int Stages = kStages;    // must be even (stage parity picks the dequantizer group)
+  static constexpr int BN = kBN;            // tokens per MMA (N)
+  static constexpr int NAcc = kNAcc;        // MMAs (token sub-tiles) sharing one dequantized weight tile
+  static constexpr int TOK = BN * NAcc;     // tokens per tile
+  static constexpr int Stages = kStages;
   static constexpr bool Bwd = kBwd;         // A = W^T (MN-major) for dX, A = W (K-major) for Y
+  // Dequantizer layout: 2 = two groups of four warps, group g expands the stages with
+  // index parity g (one lane per 64-block); 1 = all eight warps on every stage (two
+  // lanes per 64-block).
+  static constexpr int Groups = kGroups;
+  static constexpr int kDeqArrivals = (kGroups == 2) ? 4 : 8;
   static constexpr int kATile = 128 * 64 * 2;
-  static constexpr int kBTile = BN * 64 * 2;
+  static constexpr int kBTile = TOK * 64 * 2;
   static constexpr int kRBytes = 4096;      // packed codes of one 128 x 64 weight tile
   static constexpr int kThreads = 14 * 32;
-  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kAccBufs = (2 * TOK <= 512) ? 2 : 1;   // double-buffer the accumulators when TMEM allows
+  static constexpr int kTmemCols = (kAccBufs * TOK <= 32) ? 32 : (kAccBufs * TOK <= 64) ? 64 : (kAccBufs * TOK <= 128) ? 128
+                                   : (kAccBufs * TOK <= 256) ? 256 : 512;
   static constexpr int kSmemBytes = Stages * (kATile + kBTile + kRBytes) + 1024 + 256;
-  static_assert(Stages % 2 == 0, "two dequantizer groups alternate stages");
-  static_assert(BN == 16 || BN == 64 || BN == 128 || BN == 256, "token tile");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(BN % 32 == 0 || BN == 16, "epilogue reads 32 columns at a time");
+  static_assert(kAccBufs * TOK <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kGroups == 1 || (kGroups == 2 && kStages % 2 == 0), "stage parity picks the group");
 };
 
 constexpr int kRasterGroup = 4;   // token tiles per raster group (L2 reuse of both operands)
@@ -153,7 +166,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::Stages; ++s) {
       mbar_init(&tma_full[s], 1);
-      mbar_init(&deq_full[s], 4);
+      mbar_init(&deq_full[s], C::kDeqArrivals);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -195,7 +208,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_arrive_expect_tx(bar, C::kRBytes + C::kBTile);
             if (C::Bwd) tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, mb * 64, kt * 64);
             else tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, kt * 32, mb * 128);
-            tma_load_2d(b_dst, &maps.act, bar, kt * 64, nb * C::BN);
+#pragma unroll
+            for (int t = 0; t < C::NAcc; ++t)
+              tma_load_2d(b_dst + t * (C::BN * 128), &maps.act, bar, kt * 64, nb * C::TOK + t * C::BN);
           } else {
             const int e = i - nmain;
             mbar_arrive_expect_tx(bar, C::kATile + C::kBTile);
@@ -205,7 +220,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             } else {
               tma_load_2d(a_dst, &maps.a2, bar, e * 64, mb * 128);
             }
-            tma_load_2d(b_dst, &maps.b2, bar, e * 64, nb * C::BN);
+#pragma unroll
+            for (int t = 0; t < C::NAcc; ++t)
+              tma_load_2d(b_dst + t * (C::BN * 128), &maps.b2, bar, e * 64, nb * C::TOK + t * C::BN);
           }
           pending |= (1u << stage);
           pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
@@ -237,7 +254,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         wdecode(p, u, mb, nb, split, kt0, nmain, next);
         if (!mbar_wait(&acc_empty[acc], aph ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::TOK);
         for (int i = 0; i < nmain + next; ++i) {
           if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
           if (!mbar_wait(&deq_full[stage], ph)) { ok = false; break; }
@@ -248,16 +265,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = C::Bwd ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
                                        : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = umma_desc_sw128(b_addr + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int t = 0; t < C::NAcc; ++t) {
+              const uint64_t bd = umma_desc_sw128(b_addr + t * (C::BN * 128) + kk * 32, 16, 1024);
+              umma_bf16(d_tmem + t * C::BN, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           umma_commit(&empty[stage]);
           if (++stage == C::Stages) { stage = 0; ph ^= 1; }
         }
         if (!ok) break;
         umma_commit(&acc_full[acc]);
-        acc ^= 1;
-        if (acc == 0) aph ^= 1;
+        if (++acc == C::kAccBufs) { acc = 0; aph ^= 1; }
       }
     }
     __syncwarp();
@@ -272,34 +291,34 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (!mbar_wait(&acc_full[acc], aph)) break;
       tc_fence_after();
       const int feat = mb * 128 + q * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::TOK);
       if (C::BN == 16) {
         uint32_t v[32];
         tmem_ld_32x32b_x16(t_row, v);
         tmem_ld_wait();
-        wstore<16>(p, split, feat, nb * C::BN, v);
+        wstore<16>(p, split, feat, nb * C::TOK, v);
       } else {
 #pragma unroll 1
-        for (int c = 0; c < C::BN / 32; ++c) {
+        for (int c = 0; c < C::TOK / 32; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(t_row + c * 32, v);
           tmem_ld_wait();
-          wstore<32>(p, split, feat, nb * C::BN + c * 32, v);
+          wstore<32>(p, split, feat, nb * C::TOK + c * 32, v);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      acc ^= 1;
-      if (acc == 0) aph ^= 1;
+      if (++acc == C::kAccBufs) { acc = 0; aph ^= 1; }
     }
-  } else {
-    // ------------------------------------------------------------ dequantizers
-    const int grp = (warp - 6) >> 2;                 // owns stages with (stage & 1) == grp
+  } else if (C::Groups == 2) {
+    // ------------------------------------------------------------ dequantizers (two groups)
+    // Group g (four warps) expands the stages with index parity g, so two K steps are in
+    // flight at once. Forward: thread = W row of the 128-row tile, one 64-block per K step.
+    // Backward: thread = (W row i of the 64-row K step, 64-column block c of the tile).
+    const int grp = (warp - 6) >> 2;
     const int gt = threadIdx.x - 192 - 128 * grp;    // 0..127
     const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
-    // Forward: thread = W row of the 128-row tile, one 64-block per K step.
-    // Backward: thread = (W row i of the 64-row K step, 64-column block c of the 128-column tile).
     const int i_mn = gt & 63;
     const int c_mn = gt >> 6;
     uint32_t r_off0, r_off1, a_off;
@@ -323,7 +342,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int mb, nb, split, kt0, nmain, next;
       wdecode(p, u, mb, nb, split, kt0, nmain, next);
-      // scale prefetch: own K steps are every other step; keep two of them in flight
       const int first = ((stage & 1) == grp) ? 0 : 1;
       auto block_of = [&](int i, bool& valid) -> int64_t {
         const int kt = kt0 + i;
@@ -333,6 +351,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
         return wrow * p.w_kblocks + kb;
       };
+      // scale prefetch: own K steps are every other step; keep two of them in flight
       RawScale r0{0u, 0.f}, r1{0u, 0.f};
       {
         bool v0, v1;
@@ -342,8 +361,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         if (first + 2 < nmain && v1) r1 = load_raw_scale(p.scales, b1);
       }
       for (int i = 0; i < nmain + next; ++i) {
-        const bool mine = ((stage & 1) == grp);
-        if (mine) {
+        if ((stage & 1) == grp) {
           if (i < nmain) {
             bool valid, v2;
             block_of(i, valid);
@@ -374,12 +392,94 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             r0 = r1;
             r1 = r2;
           } else {
-            // extension step: the producer loads the A tile; keep the phases in step
             if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&deq_full[stage]);
         }
+        if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dequantizers (all warps)
+    // 256 threads per K step. Forward: thread = (W row r of the 128-row tile, half h of
+    // its 64-block). Backward: thread = (W row i of the 64-row K step, 64-column block c
+    // of the 128-column tile, half h).
+    const int gt = threadIdx.x - 192;                 // 0..255
+    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
+    int row_f = 0, i_mn = 0, c_mn = 0, h;
+    uint32_t r_off, a_off;
+    int sw;
+    if (!C::Bwd) {
+      row_f = gt >> 1;
+      h = gt & 1;
+      const uint32_t x = (row_f >> 2) & 1;                  // 32B swizzle of the code tile
+      r_off = row_f * 32 + 16 * (h ^ x);
+      a_off = (row_f >> 3) * 1024 + (row_f & 7) * 128;
+      sw = row_f & 7;
+    } else {
+      i_mn = gt & 63;
+      c_mn = (gt >> 6) & 1;
+      h = gt >> 7;
+      const uint32_t x = (i_mn >> 1) & 3;                   // 64B swizzle of the code tile
+      r_off = i_mn * 64 + 16 * ((2 * c_mn + h) ^ x);
+      a_off = c_mn * 8192 + (i_mn >> 3) * 1024 + (i_mn & 7) * 128;
+      sw = i_mn & 7;
+    }
+    int stage = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int mb, nb, split, kt0, nmain, next;
+      wdecode(p, u, mb, nb, split, kt0, nmain, next);
+      auto block_of = [&](int i, bool& valid) -> int64_t {
+        const int kt = kt0 + i;
+        int64_t wrow, kb;
+        if (!C::Bwd) { wrow = static_cast<int64_t>(mb) * 128 + row_f; kb = kt; }
+        else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(mb) * 2 + c_mn; }
+        valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
+        return wrow * p.w_kblocks + kb;
+      };
+      // scale prefetch: two K steps ahead
+      RawScale r0{0u, 0.f}, r1{0u, 0.f};
+      {
+        bool v0, v1;
+        const int64_t b0 = block_of(0, v0);
+        const int64_t b1 = block_of(1, v1);
+        if (0 < nmain && v0) r0 = load_raw_scale(p.scales, b0);
+        if (1 < nmain && v1) r1 = load_raw_scale(p.scales, b1);
+      }
+      for (int i = 0; i < nmain + next; ++i) {
+        if (i < nmain) {
+          bool valid, v2;
+          block_of(i, valid);
+          const int64_t b2 = block_of(i + 2, v2);
+          RawScale r2{0u, 0.f};
+          if (i + 2 < nmain && v2) r2 = load_raw_scale(p.scales, b2);
+          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
+          const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
+          if (valid) {
+            const uint4 w = ld_shared_v4_w(smem_u32(sR + stage * C::kRBytes) + r_off);
+            const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales, r0, mean));
+            const int j0 = 4 * h;
+            st_shared_v4_w(adst + (((j0 + 0) ^ sw) << 4), nf4_lookup8(lut, w.x));
+            st_shared_v4_w(adst + (((j0 + 1) ^ sw) << 4), nf4_lookup8(lut, w.y));
+            st_shared_v4_w(adst + (((j0 + 2) ^ sw) << 4), nf4_lookup8(lut, w.z));
+            st_shared_v4_w(adst + (((j0 + 3) ^ sw) << 4), nf4_lookup8(lut, w.w));
+          } else {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st_shared_v4_w(adst + ((4 * h + j) << 4), z);
+          }
+          fence_proxy_async_smem();
+          r0 = r1;
+          r1 = r2;
+        } else {
+          // extension step: the producer loads the A tile; keep the phases in step
+          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&deq_full[stage]);
         if (++stage == C::Stages) { stage = 0; ph ^= 1; }
       }
     }
@@ -413,6 +513,8 @@ static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid,
   return cudaGetLastError();
 }
 
+int wgemm_box_rows(int bn) { return bn == 384 ? 192 : bn; }
+
 int wgemm_bn(int64_t tokens) {
   if (tokens <= 16) return 16;
   if (tokens <= 64) return 64;
@@ -427,17 +529,17 @@ cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& map
   cudaError_t e = cudaErrorInvalidValue;
   if (!bwd) {
     switch (bn) {
-      case 16: e = launch_wcfg<WCfg<16, 8, false>>(p, maps, grid, st); break;
-      case 64: e = launch_wcfg<WCfg<64, 8, false>>(p, maps, grid, st); break;
-      case 128: e = launch_wcfg<WCfg<128, 6, false>>(p, maps, grid, st); break;
-      case 256: e = launch_wcfg<WCfg<256, 4, false>>(p, maps, grid, st); break;
+      case 16: e = launch_wcfg<WCfg<16, 1, 8, false>>(p, maps, grid, st); break;
+      case 64: e = launch_wcfg<WCfg<64, 1, 8, false>>(p, maps, grid, st); break;
+      case 128: e = launch_wcfg<WCfg<128, 1, 6, false>>(p, maps, grid, st); break;
+      case 256: e = launch_wcfg<WCfg<256, 1, 4, false>>(p, maps, grid, st); break;
     }
   } else {
     switch (bn) {
-      case 16: e = launch_wcfg<WCfg<16, 8, true>>(p, maps, grid, st); break;
-      case 64: e = launch_wcfg<WCfg<64, 8, true>>(p, maps, grid, st); break;
-      case 128: e = launch_wcfg<WCfg<128, 6, true>>(p, maps, grid, st); break;
-      case 256: e = launch_wcfg<WCfg<256, 4, true>>(p, maps, grid, st); break;
+      case 16: e = launch_wcfg<WCfg<16, 1, 8, true>>(p, maps, grid, st); break;
+      case 64: e = launch_wcfg<WCfg<64, 1, 8, true>>(p, maps, grid, st); break;
+      case 128: e = launch_wcfg<WCfg<128, 1, 6, true>>(p, maps, grid, st); break;
+      case 256: e = launch_wcfg<WCfg<256, 1, 4, true>>(p, maps, grid, st); break;
     }
   }
   if (timed) timing_record(st, false, algo_flops);

@@ -26,6 +26,25 @@ size_t g_events_used = 0;
 }  // namespace
 
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+Nf4Buckets nf4_buckets_from_midpoints(const float* mid) {
+  // Widened buckets [(b-1)/16 - 1 - eps, b/16 - 1 + eps]: neighbouring thresholds are
+  // >= 0.08 apart, wider than a widened bucket, so each holds at most one.
+  const double eps = 1e-3;
+  Nf4Buckets bk;
+  for (int b = 0; b < 35; ++b) {
+    const double lo = (b - 1) / 16.0 - 1.0 - eps, hi = b / 16.0 - 1.0 + eps;
+    int below = 0;
+    float thr = INFINITY;
+    for (int i = 0; i < 15; ++i) {
+      if (static_cast<double>(mid[i]) < lo) ++below;
+      else if (static_cast<double>(mid[i]) <= hi) thr = mid[i];
+    }
+    bk.base[b] = below;
+    bk.thr[b] = thr;
+  }
+  return bk;
+}
 bool timing_active() { return g_timing_on.load(std::memory_order_relaxed); }
 
 void timing_record(cudaStream_t st, bool start, double flops) {
@@ -92,6 +111,11 @@ Nf4Table build_table() {
 const Nf4Table& table() {
   static const Nf4Table t = build_table();
   return t;
+}
+
+const Nf4Buckets& buckets() {
+  static const Nf4Buckets b = qlora::nf4_buckets_from_midpoints(table().mid);
+  return b;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -201,6 +225,7 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   part = std::max(part, static_cast<size_t>(P.db.splits) * n * rp);
   part = std::max(part, static_cast<size_t>(P.da.splits) * k * rp);
   if (P.fwd.splits > 1) part = std::max(part, static_cast<size_t>(P.fwd.splits) * m * n);
+  if (m <= 64) part = std::max(part, static_cast<size_t>(lora_down_small_slices(k)) * m * rp);
   if (P.bwd.splits > 1) part = std::max(part, static_cast<size_t>(P.bwd.splits) * m * k);
   P.off_part = take(part * 4);
   P.total = off;
@@ -336,7 +361,7 @@ int qlora_nf4_quantize(const float* W, qlora_nf4_weight* w, void* ws, size_t ws_
     if (ws == nullptr || !aligned16(ws) || ws_bytes < quant_ws_layout(n_elem).total) return QLORA_ERR_WORKSPACE;
   }
   const cudaError_t e =
-      launch_quantize(W, n_elem, table(), w->codes, dq ? nullptr : w->scale_bf16, dq ? w->scale_fp8 : nullptr,
+      launch_quantize(W, n_elem, table(), buckets(), w->codes, dq ? nullptr : w->scale_bf16, dq ? w->scale_fp8 : nullptr,
                       dq ? w->dq_scale : nullptr, dq ? w->dq_mean : nullptr, ws, num_sms(),
                       reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e);
@@ -371,8 +396,14 @@ int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, co
   uint16_t* sU = reinterpret_cast<uint16_t*>(wsb + P.off_scaled);
 
   // U = X A^T (fp32, optionally saved) and bf16(s * U) for the K extension
-  int rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st);
-  if (rc != QLORA_OK) return rc;
+  if (m <= 64) {
+    if (launch_lora_down_small(X, m, k, A, r, P.r_pad, s, U_save, sU, reinterpret_cast<float*>(wsb + P.off_part),
+                               st) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+  } else {
+    const int rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st);
+    if (rc != QLORA_OK) return rc;
+  }
 
   // Y^T = W . X^T + B . (sU)^T with W dequantized on the fly (weight as the 128-row operand)
   GemmParams p = base_params(n, m, P.bn, k / 64, P.fwd);
@@ -391,11 +422,11 @@ int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, co
   }
   WMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  bool ok = map_bf16(&maps.act, X, m, k, static_cast<uint32_t>(P.bn));
+  bool ok = map_bf16(&maps.act, X, m, k, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
   ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
                      static_cast<uint64_t>(k / 2), 32, 128, 32);
   ok = ok && tmap_2d(&maps.a2, B, kBF16, r, n, r * 2, 64, 128, 128);
-  ok = ok && map_bf16(&maps.b2, sU, m, P.r_pad, static_cast<uint32_t>(P.bn));
+  ok = ok && map_bf16(&maps.b2, sU, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
   if (!ok) return QLORA_ERR_CUDA;
   const double fwd_flops = 2.0 * double(m) * double(n) * double(k + r);
   cudaError_t e = launch_wgemm(false, P.bn, p, maps, grid_of(p), st, fwd_flops);
@@ -463,11 +494,11 @@ int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_
     }
     WMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    bool ok = map_bf16(&maps.act, dY, m, n, static_cast<uint32_t>(P.bn));
+    bool ok = map_bf16(&maps.act, dY, m, n, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
     ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
                        static_cast<uint64_t>(k / 2), 64, 64, 64);
     ok = ok && tmap_2d(&maps.a2, A, kBF16, k, r, k * 2, 64, 64, 128);
-    ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(P.bn));
+    ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
     if (!ok) return QLORA_ERR_CUDA;
     const double dx_flops = 2.0 * double(m) * double(k) * double(n + r);
     if (launch_wgemm(true, P.bn, p, maps, grid_of(p), st, dx_flops) != cudaSuccess) return QLORA_ERR_CUDA;

@@ -20,6 +20,15 @@ struct Nf4Table {
   float mid[16];
 };
 
+// Exact one-comparison code search for the quantizer: 35 buckets of width
+// 1/16, bucket b = [(b - 1)/16 - 1, b/16 - 1), each widened by 1e-3; thr[b]
+// is the single decision threshold inside widened bucket b (+inf if none)
+// and base[b] the number of thresholds below it. code(x) = base[b] + (x > thr[b]).
+struct Nf4Buckets {
+  float thr[35];
+  int32_t base[35];
+};
+
 // Device error word: kernels write a non-zero code here when a bounded wait
 // gives up, so the host can read the failure instead of the GPU hanging.
 enum : int { kErrNone = 0, kErrWaitTimeout = 1 };
@@ -119,6 +128,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// Contiguous bulk copy global -> shared (TMA engine, no tensor map, no
+// multicast). Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -18,7 +18,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline QuantWsLayout quant_ws_layout(int64_t n_elem) {
   const int64_t nblk = (n_elem + 63) / 64;
-  const int64_t pa = (nblk + 511) / 512;
+  const int64_t pa = (nblk + 127) / 128;          // one fp64 partial per 128 blocks
   const int64_t pb = (pa + 511) / 512 + 1;
   QuantWsLayout L;
   L.absmax_off = 0;
@@ -29,19 +29,19 @@ inline QuantWsLayout quant_ws_layout(int64_t n_elem) {
   return L;
 }
 
-cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab, uint8_t* codes,
-                            uint16_t* scale_bf16, uint8_t* scale_fp8, float* dq_scale, float* dq_mean,
-                            void* ws, int num_sms, cudaStream_t st);
+cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab, const Nf4Buckets& bk,
+                            uint8_t* codes, uint16_t* scale_bf16, uint8_t* scale_fp8, float* dq_scale,
+                            float* dq_mean, void* ws, int num_sms, cudaStream_t st);
+// Bucket table of the quantizer's code search, built from the 15 midpoints (qlora_abi.cu).
+Nf4Buckets nf4_buckets_from_midpoints(const float* mid);
 cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t n_elem, const Nf4Table& tab,
                               uint16_t* out, int num_sms, cudaStream_t st);
 
 // --------------------------------------------------------------------- GEMM
-// Operand sources of the tensor-core GEMM D[rows, cols] = sum_k A[row, k] B[col, k].
+// Operand sources of the low-rank tensor-core GEMM D[rows, cols] = sum_k A[row, k] B[col, k].
 enum BMode : int {
   kB_TmaK = 0,    // bf16 [cols, K] row-major via TMA (K-major)
   kB_TmaMN = 1,   // bf16 [K, cols] row-major via TMA (MN-major)
-  kB_Nf4K = 2,    // NF4 weight W[cols, K], dequantized in shared memory (forward)
-  kB_Nf4MN = 3,   // NF4 weight W[K, cols], dequantized in shared memory (backward dX)
 };
 
 enum OutMode : int {
@@ -56,7 +56,7 @@ struct GemmParams {
   int32_t k_tiles;             // main-loop 64-wide K steps
   int32_t ext_tiles;           // extra K steps from the second operand pair (low-rank branch)
   int32_t splits, k_per_split; // split of the main K steps
-  // NF4 operand
+  // NF4 operand (weight-operand GEMM only)
   ScaleSrc scales;
   int64_t w_kblocks;           // 64-blocks per row of W
   int32_t w_rows;              // rows of W
@@ -70,17 +70,15 @@ struct GemmParams {
 };
 
 struct GemmMaps {
-  CUtensorMap a, b, a2, b2;    // b = codes for NF4 modes; b2 = lo half for hi/lo mode
+  CUtensorMap a, b, a2, b2;    // b2 = lo half of B in the hi/lo mode (a2 unused)
 };
 
 // Host helpers (nf4_gemm.cu). swizzle: 0 none, 32, 64 or 128 (bytes).
 bool tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle);
 
-// Launch variants
+// Launch variants of the low-rank GEMM
 enum GemmKind : int {
-  kGemmFwd = 0,        // A = X (K-major), B = NF4 K-major, ext: [s*U | B_lora]
-  kGemmBwdDx = 1,      // A = dY (K-major), B = NF4 MN-major, ext: [s*G | A_lora]
   kGemmLoraDownK = 2,  // A K-major, B K-major, BN = 64 (U = X A^T)
   kGemmLoraDownMN = 3, // A K-major, B MN-major, BN = 64 (G = dY B)
   kGemmLoraGrad = 4,   // A MN-major, B MN-major hi+lo, BN = 64 (dB, dA^T)
@@ -90,9 +88,7 @@ enum GemmKind : int {
 };
 
 int gemm_bn(GemmKind kind);
-// algo_flops: algorithmic flops of this launch, used only by the optional timing hook
-cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st,
-                        double algo_flops = 0.0);
+cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st);
 
 // Launch accounting (qlora_abi.cu): every kernel launch is counted; fused NF4
 // GEMM launches can additionally be bracketed by timing events.
@@ -111,7 +107,8 @@ struct WMaps {
   CUtensorMap a2;      // low-rank A-side tile: B_lora [n, r] (forward) or A_lora [r, k] (backward)
   CUtensorMap b2;      // low-rank B-side tile: s*U or s*G [tokens, r_pad]
 };
-int wgemm_bn(int64_t tokens);
+int wgemm_bn(int64_t tokens);          // tokens per tile
+int wgemm_box_rows(int bn);              // token rows per TMA box / MMA (the tile may hold two)
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
                          double algo_flops);
 
@@ -128,6 +125,13 @@ cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_str
 cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_stride, int64_t rows,
                                  int64_t cols, int64_t ld_part, void* out, int out_bf16, int accumulate,
                                  cudaStream_t st);
+// U = X A^T on CUDA cores for a few tokens (m <= 64): fp32 U [m, r] (nullable) and
+// bf16(scale * U) [m, r_pad] (padding columns zeroed), via K-slice partials.
+// part: workspace of lora_down_small_slices(k) * m * r_pad floats for the K-slice partials.
+int lora_down_small_slices(int64_t k);
+cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
+                                   int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
+                                   cudaStream_t st);
 cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
                                  cudaStream_t st);
 cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,

@@ -77,7 +77,8 @@ extern "C" int qlora_nf4_quantize_noalloc(const float* W, qlora_nf4_weight* w, q
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return QLORA_ERR_CUDA;
-  const cudaError_t e = qlora::launch_quantize(W, n_elem, tab, w->codes, dq ? nullptr : w->scale_bf16,
+  const qlora::Nf4Buckets bk = qlora::nf4_buckets_from_midpoints(tab.mid);
+  const cudaError_t e = qlora::launch_quantize(W, n_elem, tab, bk, w->codes, dq ? nullptr : w->scale_bf16,
                                                dq ? w->scale_fp8 : nullptr, dq ? w->dq_scale : nullptr,
                                                dq ? w->dq_mean : nullptr, scratch, sms,
                                                reinterpret_cast<cudaStream_t>(stream));
