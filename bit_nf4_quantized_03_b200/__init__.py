@@ -34,7 +34,7 @@ EXPORTED = (
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_check_device_error",
     "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end",
-    "qlora_nf4_quantize_noalloc",
+    "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout",
 )
 
 
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         "qlora_timing_begin": (ctypes.c_int, [i32]),
         "qlora_timing_end": (ctypes.c_int, [vp, vp, vp]),
         "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
+        "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -218,6 +219,10 @@ def qlora_silu_gate_fwd(g, u, h, stream=None):
 def qlora_silu_gate_bwd(dh, g, u, dg, du, stream=None):
     _check(lib().qlora_silu_gate_bwd(_ptr(dh), _ptr(g), _ptr(u), _ptr(dg), _ptr(du), g.numel(), _stream(stream)),
            "qlora_silu_gate_bwd")
+
+
+def qlora_selftest_wait_timeout(limit_ms: int = 100, stream=None) -> None:
+    _check(lib().qlora_selftest_wait_timeout(int(limit_ms), _stream(stream)), "qlora_selftest_wait_timeout")
 
 
 def qlora_check_device_error(stream=None) -> None:

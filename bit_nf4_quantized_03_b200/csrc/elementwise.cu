@@ -212,6 +212,31 @@ cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, cons
 }
 
 // ---------------------------------------------------------------------------
+// Self-test of the failure path: one thread waits on an mbarrier that nothing
+// ever arrives on, with a short limit; the wait gives up, records the device
+// error word and the kernel returns normally.
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  const uint32_t a = smem_u32(&bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, 0)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicExch(&g_device_error, kErrWaitTimeout);
+      return;
+    }
+  }
+}
+
+cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st) {
+  selftest_wait_timeout_kernel<<<1, 1, 0, st>>>(limit_ns);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // SiLU-gated glue: h = silu(g) * u ; dg = dh*u*sig*(1 + g*(1-sig)), du = dh*g*sig
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }

@@ -48,6 +48,77 @@ __device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2* tab) 
   return static_cast<uint32_t>(__float_as_int(e.y)) + ((x > e.x) ? 1u : 0u);
 }
 
+__device__ __forceinline__ uint32_t bfi4(uint32_t word, uint32_t code, uint32_t pos) {
+  uint32_t d;
+  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(d) : "r"(code), "r"(word), "r"(pos));
+  return d;
+}
+
+// Codes of one lane's eight weights (x = w * inv); the first four (lo) go to
+// nibbles 0..3 of the 16-bit result, the next four (hi) to nibbles 4..7.
+__device__ __forceinline__ uint32_t nf4_codes8(const float4& lo, const float4& hi, float inv, const float2* tab) {
+  uint32_t w = 0;
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(lo.x, inv), tab), 0);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(lo.y, inv), tab), 4);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(lo.z, inv), tab), 8);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(lo.w, inv), tab), 12);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(hi.x, inv), tab), 16);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(hi.y, inv), tab), 20);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(hi.z, inv), tab), 24);
+  w = bfi4(w, nf4_code_bucket(__fmul_rn(hi.w, inv), tab), 28);
+  return w;
+}
+
+__device__ __forceinline__ float absmax8(const float4& a, const float4& b) {
+  return fmaxf(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))),
+               fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+}
+
+// Fixed pairwise tree (fp64) over part[0..n) zero-padded to a power of two,
+// by one CTA of 256 threads. Each warp reduces an aligned group of 512: every
+// lane sums its 16 consecutive values pairwise, then five xor-shuffle levels
+// combine neighbouring lanes (a + b == b + a exactly, so this is the same
+// tree). Level by level, ping-ponging between `part` and `other`, until one
+// value is left.
+__device__ double tree_sum_cta(double* part, double* other, int64_t n) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double* src = part;
+  double* dst = other;
+  while (n > 1) {
+    const int64_t groups = (n + 511) / 512;
+    for (int64_t g = warp; g < groups; g += 8) {
+      double v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t idx = g * 512 + lane * 16 + j;
+        v[j] = (idx < n) ? __ldcg(src + idx) : 0.0;           // other CTAs' sums: read through L2
+      }
+#pragma unroll
+      for (int w = 1; w < 16; w <<= 1)
+#pragma unroll
+        for (int j = 0; j < 16; j += 2 * w) v[j] = v[j] + v[j + w];
+      double t = v[0];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
+      if (lane == 0) dst[g] = t;
+    }
+    __threadfence_block();
+    __syncthreads();
+    double* sw = src;
+    src = dst;
+    dst = sw;
+    n = groups;
+  }
+  return __ldcg(src);
+}
+
+// Mean of all block absmax values from the per-chunk fp64 sums (one CTA).
+__global__ void __launch_bounds__(256) dq_mean_kernel(double* __restrict__ part, double* __restrict__ other,
+                                                      int64_t nchunks, int64_t nblk, float* __restrict__ mean_out) {
+  const double S = tree_sum_cta(part, other, nchunks);
+  if (threadIdx.x == 0) *mean_out = static_cast<float>(S / static_cast<double>(nblk));
+}
+
 template <bool kDQ>
 __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __restrict__ W, int64_t n_elem,
                                                               Nf4Buckets bk, uint8_t* __restrict__ codes,
@@ -67,7 +138,7 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
   const int64_t nchunks = (nblk + kQChunk - 1) / kQChunk;
   const int64_t my_n = (nchunks > blockIdx.x) ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   if (tid < 64) {
-    // entry b covers [(b - 1)/16 - 1, b/16 - 1); entries 0 and 34 are the padding buckets
+    // entry b covers [(b - 1)/16 - 1, b/16 - 1); entries 35.. are never indexed
     const int b = tid;
     s_tab[b] = (b < 35) ? make_float2(bk.thr[b], __int_as_float(bk.base[b]))
                         : make_float2(__int_as_float(0x7f800000), __int_as_float(15));
@@ -91,59 +162,65 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
   };
   if (tid == 0)
     for (int64_t i = 0; i < my_n && i < kQStages; ++i) issue(i);
-  const uint32_t x = (l >> 2) & 1;   // which half of its 32 bytes a lane reads first (bank-conflict free)
+  // Lanes 4..7 of a group read the second half of their 32 bytes first, so the
+  // eight lanes of a quarter-warp hit eight different bank groups.
+  const uint32_t x = (l >> 2) & 1;
+  const uint32_t sh_first = 16 * x, sh_second = 16 * (x ^ 1);
   for (int64_t i = 0; i < my_n; ++i) {
     const int st = static_cast<int>(i % kQStages);
     if (!mbar_wait(&full[st], static_cast<uint32_t>((i / kQStages) & 1))) break;
     const int64_t b0 = (blockIdx.x + i * gridDim.x) * kQChunk;
-    const uint32_t sbase = smem_u32(q_stage + st * (kQChunk * 256));
+    const uint32_t sbase = smem_u32(q_stage + st * (kQChunk * 256)) + l * 32;
+    const bool whole = (b0 + kQChunk <= nfull);
 #pragma unroll 2
     for (int it = 0; it < kQChunk / 32; ++it) {
       const int lb = it * 32 + grp;
       const int64_t b = b0 + lb;
-      float v[8];
-      if (b < nfull) {
-        const uint32_t src = sbase + lb * 256 + l * 32;
-        float4 h0, h1;
+      uint32_t word;
+      float m;
+      if (whole || b < nfull) {
+        float4 f, g;   // f: elements of the half read first, g: the other half
+        const uint32_t src = sbase + lb * 256;
         asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(h0.x), "=f"(h0.y), "=f"(h0.z), "=f"(h0.w) : "r"(src + 16 * x) : "memory");
+                     : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(src + sh_first) : "memory");
         asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(h1.x), "=f"(h1.y), "=f"(h1.z), "=f"(h1.w) : "r"(src + 16 * (x ^ 1)) : "memory");
-        const float4 lo = x ? h1 : h0;
-        const float4 hi = x ? h0 : h1;
-        v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
-        v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int64_t idx = 8 * l + e;
-          v[e] = (b == nfull && idx < tail) ? W[b * 64 + idx] : 0.f;
+                     : "=f"(g.x), "=f"(g.y), "=f"(g.z), "=f"(g.w) : "r"(src + sh_second) : "memory");
+        m = absmax8(f, g);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        word = 0x77777777u;               // zero or subnormal absmax: the exact-zero level
+        if (m >= 1.17549435e-38f) {
+          const uint32_t w = nf4_codes8(f, g, __frcp_rn(m), s_tab);   // f -> nibbles 0..3, g -> 4..7
+          word = x ? ((w << 16) | (w >> 16)) : w;                    // back to element order
         }
-      }
-      float m = fabsf(v[0]);
-#pragma unroll
-      for (int e = 1; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      uint32_t word = 0x77777777u;      // zero or subnormal absmax: the exact-zero level
-      if (m >= 1.17549435e-38f) {
-        const float inv = __frcp_rn(m);
-        word = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) word |= nf4_code_bucket(__fmul_rn(v[e], inv), s_tab) << (4 * e);
-      }
-      if (b < nfull) {
         reinterpret_cast<uint32_t*>(codes)[b * 8 + l] = word;
-      } else if (b == nfull && tail > 0) {
-        // ragged last block: only the bytes that hold present elements; an odd tail keeps its high nibble 0
+      } else {
+        float4 f, g;
+        float* fv = reinterpret_cast<float*>(&f);
+        float* gv = reinterpret_cast<float*>(&g);
 #pragma unroll
-        for (int byte = 0; byte < 4; ++byte) {
-          const int64_t e0 = 8 * l + 2 * byte;
-          if (e0 < tail) {
-            uint32_t c = (word >> (8 * byte)) & 0xFFu;
-            if (e0 + 1 >= tail) c &= 0x0Fu;
-            codes[b * 32 + 4 * l + byte] = static_cast<uint8_t>(c);
+        for (int e = 0; e < 4; ++e) {
+          const int64_t i0 = 8 * l + e, i1 = 8 * l + 4 + e;
+          fv[e] = (b == nfull && i0 < tail) ? W[b * 64 + i0] : 0.f;
+          gv[e] = (b == nfull && i1 < tail) ? W[b * 64 + i1] : 0.f;
+        }
+        m = absmax8(f, g);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        word = 0x77777777u;
+        if (m >= 1.17549435e-38f) word = nf4_codes8(f, g, __frcp_rn(m), s_tab);
+        if (b == nfull && tail > 0) {
+          // ragged last block: only the bytes that hold present elements; an odd tail keeps its high nibble 0
+#pragma unroll
+          for (int byte = 0; byte < 4; ++byte) {
+            const int64_t e0 = 8 * l + 2 * byte;
+            if (e0 < tail) {
+              uint32_t c = (word >> (8 * byte)) & 0xFFu;
+              if (e0 + 1 >= tail) c &= 0x0Fu;
+              codes[b * 32 + 4 * l + byte] = static_cast<uint8_t>(c);
+            }
           }
         }
       }
@@ -169,32 +246,6 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
       __syncthreads();
     }
     if (tid == 0 && i + kQStages < my_n) issue(i + kQStages);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Fixed-order fp64 sum of the absmax values: a pairwise tree over the array
-// zero-padded to a power of two. Each pass reduces aligned chunks of 512 to
-// one value with the same tree shape, so chaining passes gives exactly the
-// tree over the padded array (adding exact zeros changes nothing).
-// ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(256) pairwise_sum_pass(const T* __restrict__ in, int64_t n_in,
-                                                          double* __restrict__ out, int64_t count_for_mean,
-                                                          float* __restrict__ mean_out) {
-  __shared__ double s[256];
-  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * 512 + 2 * threadIdx.x;
-  const double a = (i0 < n_in) ? static_cast<double>(in[i0]) : 0.0;
-  const double b = (i0 + 1 < n_in) ? static_cast<double>(in[i0 + 1]) : 0.0;
-  s[threadIdx.x] = a + b;
-  __syncthreads();
-  for (int stride = 1; stride < 256; stride <<= 1) {
-    if ((threadIdx.x & (2 * stride - 1)) == 0) s[threadIdx.x] = s[threadIdx.x] + s[threadIdx.x + stride];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    out[blockIdx.x] = s[0];
-    if (mean_out != nullptr) *mean_out = static_cast<float>(s[0] / static_cast<double>(count_for_mean));
   }
 }
 
@@ -272,13 +323,21 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
   if (tid == 0)
     for (int64_t i = 0; i < my_n && i < kDStages; ++i) issue(i);
   const uint32_t x = (lane >> 2) & 1;           // read order that keeps the two 16-byte loads conflict-free
+  // the scale of this lane's block in the next chunk is loaded one chunk ahead
+  float c_next = 0.f;
+  {
+    const int64_t bn = static_cast<int64_t>(blockIdx.x) * kDChunk + warp * 32 + lane;
+    if (my_n > 0 && bn < nfull) c_next = block_scale(ss, bn, mean);
+  }
   for (int64_t i = 0; i < my_n; ++i) {
     const int st = static_cast<int>(i % kDStages);
     const int64_t b0 = (blockIdx.x + i * gridDim.x) * kDChunk + warp * 32;
     const int64_t b = b0 + lane;
-    // scale loads go out before the wait so their latency overlaps it
-    float c = 0.f;
-    if (b < nfull) c = block_scale(ss, b, mean);
+    const float c = c_next;
+    {
+      const int64_t bn = b + static_cast<int64_t>(gridDim.x) * kDChunk;
+      if (i + 1 < my_n && bn < nfull) c_next = block_scale(ss, bn, mean);
+    }
     if (!mbar_wait(&full[st], static_cast<uint32_t>((i / kDStages) & 1))) break;
     if (b < nfull) {
       const uint32_t src = smem_u32(ring + st * (kDChunk * 32) + (warp * 32 + lane) * 32);
@@ -374,28 +433,18 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   double* part_a = reinterpret_cast<double*>(static_cast<char*>(ws) + L.part_a_off);
   double* part_b = reinterpret_cast<double*>(static_cast<char*>(ws) + L.part_b_off);
   float* mean_tmp = reinterpret_cast<float*>(static_cast<char*>(ws) + L.mean_off);
-  // stage 1 also writes one fp64 tree sum per 128 blocks (the first levels of the fixed-order sum)
+  // stage 1 also writes one fp64 tree sum per chunk (the first levels of the fixed-order sum)
   e = set_smem_once(nf4_quantize_kernel<true>, kQSmem, smem_set[1]);
   if (e != cudaSuccess) return e;
   nf4_quantize_kernel<true><<<grid, 256, kQSmem, st>>>(W, n_elem, bk, codes, nullptr, absmax, part_a);
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // remaining levels: aligned chunks of 512 -> 1 until one value is left, then the mean
-  double* src = part_a;
-  double* dst = part_b;
-  int64_t n = nchunks;
-  do {
-    const int64_t g = (n + 511) / 512;
-    pairwise_sum_pass<double><<<static_cast<int>(g), 256, 0, st>>>(src, n, dst, nblk, g == 1 ? mean_tmp : nullptr);
-    count_launches(1);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    double* t = src;
-    src = dst;
-    dst = t;
-    n = g;
-  } while (n > 1);
+  // the rest of the tree and the mean
+  dq_mean_kernel<<<1, 256, 0, st>>>(part_a, part_b, nchunks, nblk, mean_tmp);
+  count_launches(1);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const int64_t nb2 = (nblk + 255) / 256;
   dq_fp8_kernel<<<static_cast<int>(nb2), 256, 0, st>>>(absmax, nblk, mean_tmp, scale_fp8, dq_scale, dq_mean);
   count_launches(1);

@@ -351,23 +351,27 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
         return wrow * p.w_kblocks + kb;
       };
-      // scale prefetch: own K steps are every other step; keep two of them in flight
-      RawScale r0{0u, 0.f}, r1{0u, 0.f};
+      // scale prefetch: own K steps are every other step; keep four of them in flight
+      RawScale r0{0u, 0.f}, r1{0u, 0.f}, r2{0u, 0.f}, r3{0u, 0.f};
       {
-        bool v0, v1;
-        const int64_t b0 = block_of(first, v0);
-        const int64_t b1 = block_of(first + 2, v1);
-        if (first < nmain && v0) r0 = load_raw_scale(p.scales, b0);
-        if (first + 2 < nmain && v1) r1 = load_raw_scale(p.scales, b1);
+        bool v;
+        int64_t bb = block_of(first, v);
+        if (first < nmain && v) r0 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 2, v);
+        if (first + 2 < nmain && v) r1 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 4, v);
+        if (first + 4 < nmain && v) r2 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 6, v);
+        if (first + 6 < nmain && v) r3 = load_raw_scale(p.scales, bb);
       }
       for (int i = 0; i < nmain + next; ++i) {
         if ((stage & 1) == grp) {
           if (i < nmain) {
-            bool valid, v2;
+            bool valid, v4;
             block_of(i, valid);
-            const int64_t b2 = block_of(i + 4, v2);
-            RawScale r2{0u, 0.f};
-            if (i + 4 < nmain && v2) r2 = load_raw_scale(p.scales, b2);
+            const int64_t b4 = block_of(i + 8, v4);
+            RawScale r4{0u, 0.f};
+            if (i + 8 < nmain && v4) r4 = load_raw_scale(p.scales, b4);
             if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
             const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
             if (valid) {
@@ -391,6 +395,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             fence_proxy_async_smem();
             r0 = r1;
             r1 = r2;
+            r2 = r3;
+            r3 = r4;
           } else {
             if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
           }

@@ -571,6 +571,12 @@ int qlora_timing_end(double* total_ms, int32_t* launches, double* flops) {
   return rc;
 }
 
+int qlora_selftest_wait_timeout(int32_t limit_ms, qlora_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return QLORA_ERR_INVALID;
+  return cuda_status(launch_selftest_wait_timeout(static_cast<uint64_t>(limit_ms) * 1000000ull,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qlora_check_device_error(qlora_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;

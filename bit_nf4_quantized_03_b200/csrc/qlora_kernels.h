@@ -132,6 +132,7 @@ int lora_down_small_slices(int64_t k);
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
                                    int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
                                    cudaStream_t st);
+cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
                                  cudaStream_t st);
 cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,

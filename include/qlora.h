@@ -209,6 +209,13 @@ int64_t qlora_launch_count(void);
 int qlora_timing_begin(int32_t max_launches);
 int qlora_timing_end(double *total_ms, int32_t *launches, double *flops);
 
+/* Exercises the failure path without faulting the GPU: launches one thread
+ * that waits on a barrier nobody arrives on and gives up after limit_ms
+ * (1..2000), recording the device error word exactly as a stuck pipeline
+ * would. The kernel then returns normally; qlora_check_device_error reports
+ * QLORA_ERR_DEVICE once and the context stays usable. */
+int qlora_selftest_wait_timeout(int32_t limit_ms, qlora_stream_t stream);
+
 /* Reads and clears the device error word (set when a kernel gave up on a
  * bounded wait). Synchronizes `stream`. Returns QLORA_OK or QLORA_ERR_DEVICE. */
 int qlora_check_device_error(qlora_stream_t stream);
