@@ -52,6 +52,13 @@ design notes of the repository):
 8. Layer: Y = X W'^T + (alpha/r) (X A^T) B^T; backward dX = dY W' +
    (alpha/r)(dY B) A, dB = (alpha/r) dY^T (X A^T), dA = (alpha/r)(dY B)^T X.
    No gradient for W' ([CSD] Piece 3: the quantized base is frozen).
+9. Adapter merge ([CSD] "Price 2: deployment friction": the adapter is
+   merged onto a dequantized BF16 copy, since a 4-bit matrix cannot absorb
+   it; [GAMUT] Step 5 "Save and Merge Adapters"; "QLoRA vs LoRA" FAQ on
+   converting back to full precision, FP16 or FP32, and quantizing again
+   for deployment): W_merged = W' + (alpha/r) B A, exact in fp64 here; the
+   stored BF16 or FP32 copy is that value rounded once (checked by the
+   tests with the bound their docstrings derive).
 """
 from __future__ import annotations
 
@@ -339,6 +346,14 @@ def linear_backward(Wd, X, dY, A, B, alpha: float, dx_rows=None):
     else:
         dX = dY @ Wd + s * (G @ A)
     return dX, dA, dB
+
+
+def lora_merge(Wd, A, B, alpha: float) -> np.ndarray:
+    """W_merged = W' + (alpha/r) B A in fp64 (reading 9): the dense weight
+    that makes the merged layer X W_merged^T equal the adapted layer."""
+    Wd, A, B = _f64(Wd), _f64(A), _f64(B)
+    s = float(alpha) / A.shape[0]
+    return Wd + s * (B @ A)
 
 
 def silu_gate_forward(g, u):

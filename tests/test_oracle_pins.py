@@ -388,3 +388,25 @@ def test_silu_gate_against_finite_differences():
     num_u = (o.silu_gate_forward(g, u + eps) - o.silu_gate_forward(g, u - eps)) / (2 * eps) * dh
     np.testing.assert_allclose(dg, num_g, rtol=1e-6, atol=1e-9)
     np.testing.assert_allclose(du, num_u, rtol=1e-6, atol=1e-9)
+
+
+def test_lora_merge_against_python_loops_and_the_layer():
+    # W_merged = W' + (alpha/r) B A ("Price 2: deployment friction": merge onto a dequantized copy)
+    Wd, X, A, B, _ = _tiny_layer(M=6, N=5, K=64, r=3)
+    alpha = 16.0
+    Wm = o.lora_merge(Wd, A, B, alpha)
+    s = alpha / 3
+    for i in range(5):
+        for j in range(64):
+            acc = float(Wd[i, j])
+            for t in range(3):
+                acc += s * float(B[i, t]) * float(A[t, j])
+            assert abs(Wm[i, j] - acc) <= 1e-15 * (1 + abs(acc)), (i, j)
+    # the merged weight reproduces the adapted layer's output
+    Y, _ = o.linear_forward(Wd, X, A, B, alpha)
+    np.testing.assert_allclose(X @ Wm.T, Y, rtol=1e-12, atol=1e-13)
+    # a freshly initialised adapter (B = 0) leaves the dequantized weight unchanged
+    assert np.array_equal(o.lora_merge(Wd, A, np.zeros_like(B), alpha), Wd)
+    # the update has rank at most r
+    sv = np.linalg.svd(Wm - Wd, compute_uv=False)
+    assert np.all(sv[3:] <= 1e-12 * sv[0])
