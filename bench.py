@@ -514,7 +514,7 @@ def run_native(args) -> None:
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
                 "frac": (achieved / peak_tc) if achieved else None, "traffic": None,
-                "kernel": "qlora_gemm_kernel (fused NF4 dequant + tcgen05, forward Y and backward dX)",
+                "kernel": "qlora_wgemm_kernel (fused NF4 dequant + tcgen05, weight as the 128-row operand; forward Y and backward dX)",
                 "launches_timed": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1),
                 "peak_kind": f"bf16_tflops_sustained ({peaks['_source']})"}
     comp = None
