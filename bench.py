@@ -404,6 +404,15 @@ def components(dev, peaks) -> dict:
     algo = n * k * (0.5 + 1.0 / 64 + 4.0 / 16384) + 2.0 * M_SMALL * (k + n) + 2.0 * RANK_R * (k + n)
     out["fwd_m16_q_proj"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
                              "algo_bytes": algo}
+    # adapter merge onto the dequantized weight (65B q_proj, bf16 output)
+    wm = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
+    fn = lambda: q.qlora_lora_merge(qw, a, b, RANK_R, ALPHA, wm, q.QLORA_DTYPE_BF16)
+    for _ in range(3):
+        fn()
+    ms = graph_time(fn, 10, flush)
+    algo = n * k * (0.5 + 1.0 / 64 + 4.0 / 16384 + 2.0) + 2.0 * RANK_R * (k + n)
+    out["merge_q_proj"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
+                           "algo_bytes": algo}
     return out
 
 
@@ -440,6 +449,16 @@ def run_case(args) -> None:
                 q.qlora_linear_bwd(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, ws)
             else:
                 q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+    elif name == "merge_q_65b":
+        n, k = LAYERS[0][1], LAYERS[0][2]
+        W = synth.weight(n, k).to(dev)
+        qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+        q.qlora_nf4_quantize(W, qw)
+        del W
+        a, b = (t.to(dev) for t in synth.lora_pair(RANK_R, k, n))
+        wm = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
+        for _ in range(1 + args.case_iters):
+            q.qlora_lora_merge(qw, a, b, RANK_R, ALPHA, wm, q.QLORA_DTYPE_BF16)
     elif name in ("quantize_4096", "dequantize_4096"):
         W = synth.weight(4096, 4096, outlier_frac=0.001).to(dev)
         qw = q.QuantizedWeight(4096, 4096, q.QLORA_SCALE_DQ_FP8, device=dev)

@@ -34,7 +34,7 @@ EXPORTED = (
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_check_device_error",
     "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end",
-    "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout",
+    "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
 )
 
 
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
         "qlora_timing_end": (ctypes.c_int, [vp, vp, vp]),
         "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
         "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
+        "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -184,6 +185,13 @@ def qlora_nf4_quantize(W: torch.Tensor, w: QuantizedWeight, ws: torch.Tensor | N
 
 def qlora_nf4_dequantize(w: QuantizedWeight, out: torch.Tensor, stream=None) -> torch.Tensor:
     _check(lib().qlora_nf4_dequantize(w.ref(), _ptr(out), _stream(stream)), "qlora_nf4_dequantize")
+    return out
+
+
+def qlora_lora_merge(w: QuantizedWeight, A, B, r: int, alpha: float, out, out_dtype: int, stream=None):
+    """out[n, k] = dequant(w) + (alpha / r) B A, in bf16 or fp32 (out_dtype)."""
+    _check(lib().qlora_lora_merge(w.ref(), _ptr(A), _ptr(B), r, alpha, _ptr(out), out_dtype, _stream(stream)),
+           "qlora_lora_merge")
     return out
 
 

@@ -96,28 +96,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 }
 
 // Raw scale of one block, loaded ahead of use; turned into the fp32 scale later.
-struct RawScale {
-  uint32_t q;
-  float s2;
-};
-
-__device__ __forceinline__ RawScale load_raw_scale(const ScaleSrc& s, int64_t b) {
-  RawScale r;
-  if (s.bf16 != nullptr) {
-    r.q = __ldg(s.bf16 + b);
-    r.s2 = 0.f;
-  } else {
-    r.q = __ldg(s.fp8 + b);
-    r.s2 = __ldg(s.dq_scale + (b >> 8));
-  }
-  return r;
-}
-
-__device__ __forceinline__ float raw_to_scale(const ScaleSrc& s, const RawScale& r, float mean) {
-  if (s.bf16 != nullptr) return __uint_as_float(r.q << 16);
-  return __fadd_rn(__fmul_rn(e4m3_to_float(static_cast<uint8_t>(r.q)), r.s2), mean);
-}
-
 // Epilogue: 32 (or 16) consecutive tokens of one output feature.
 template <int kCount>
 __device__ __forceinline__ void wstore(const GemmParams& p, int split, int feat, int tok0, const uint32_t (&v)[32]) {

@@ -379,6 +379,40 @@ size_t qlora_linear_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) 
   return make_plan(m, n, k, r).total;
 }
 
+int qlora_lora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int32_t r, float alpha,
+                     void* W_out, int32_t out_dtype, qlora_stream_t stream) {
+  if (!weight_ok(w) || A == nullptr || B == nullptr || W_out == nullptr) return QLORA_ERR_INVALID;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(W_out)) return QLORA_ERR_INVALID;
+  if (out_dtype != QLORA_DTYPE_BF16 && out_dtype != QLORA_DTYPE_FP32) return QLORA_ERR_INVALID;
+  if (w->k % 64 != 0 || !(r == 8 || r == 16 || r == 32 || r == 64 || r == 128)) return QLORA_ERR_UNSUPPORTED;
+  const int64_t n = w->n, k = w->k;
+  const int64_t tiles_m = cdiv(n, 128), tiles_n = cdiv(k, merge_tile_cols());
+  if (tiles_m * tiles_n > INT32_MAX) return QLORA_ERR_UNSUPPORTED;
+  MergeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tiles_m = static_cast<int32_t>(tiles_m);
+  p.tiles_n = static_cast<int32_t>(tiles_n);
+  p.k_steps = static_cast<int32_t>(cdiv(r, 64));
+  p.n = n;
+  p.k = k;
+  p.codes = w->codes;
+  p.scales = scale_src(w);
+  p.scale = alpha / static_cast<float>(r);
+  p.out = W_out;
+  p.tab = table();
+  const bool f32 = (out_dtype == QLORA_DTYPE_FP32);
+  MergeMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  bool ok = tmap_2d(&maps.b, B, kBF16, r, n, r * 2, 64, 128, 128);
+  ok = ok && tmap_2d(&maps.a, A, kBF16, k, r, k * 2, 64, 64, 128);
+  ok = ok && tmap_2d(&maps.codes, w->codes, kU8, k / 2, n, k / 2, 128, 128, 128);
+  ok = ok && (f32 ? tmap_2d(&maps.out, W_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, k, n, k * 4, 32, 32, 128)
+                  : tmap_2d(&maps.out, W_out, kBF16, k, n, k * 2, 32, 32, 64));
+  if (!ok) return QLORA_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles_m * tiles_n, num_sms()));
+  return cuda_status(launch_merge(p, maps, grid, f32, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, const uint16_t* A, const uint16_t* B,
                      int32_t r, float alpha, void* Y, int32_t y_dtype, float* U_save, void* ws, size_t ws_bytes,
                      qlora_stream_t stream) {

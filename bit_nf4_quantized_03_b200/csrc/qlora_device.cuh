@@ -139,6 +139,26 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
                : "memory");
 }
 
+// Tiled store shared -> global through the TMA engine (bulk-group completion).
+// Elements outside the tensor are not written. x must be 16-byte aligned.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N committed bulk groups are still in flight (writes complete).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -299,6 +319,30 @@ __device__ __forceinline__ float block_scale(const ScaleSrc& s, int64_t b, float
   }
   const float q = e4m3_to_float(__ldg(s.fp8 + b));
   return __fadd_rn(__fmul_rn(q, __ldg(s.dq_scale + (b >> 8))), mean);
+}
+
+// Raw scale bytes of one block, loaded ahead of use; raw_to_scale gives the
+// same fp32 value as block_scale.
+struct RawScale {
+  uint32_t q;
+  float s2;
+};
+
+__device__ __forceinline__ RawScale load_raw_scale(const ScaleSrc& s, int64_t b) {
+  RawScale r;
+  if (s.bf16 != nullptr) {
+    r.q = __ldg(s.bf16 + b);
+    r.s2 = 0.f;
+  } else {
+    r.q = __ldg(s.fp8 + b);
+    r.s2 = __ldg(s.dq_scale + (b >> 8));
+  }
+  return r;
+}
+
+__device__ __forceinline__ float raw_to_scale(const ScaleSrc& s, const RawScale& r, float mean) {
+  if (s.bf16 != nullptr) return __uint_as_float(r.q << 16);
+  return __fadd_rn(__fmul_rn(e4m3_to_float(static_cast<uint8_t>(r.q)), r.s2), mean);
 }
 
 }  // namespace qlora

@@ -112,6 +112,27 @@ int wgemm_box_rows(int bn);              // token rows per TMA box / MMA (the ti
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
                          double algo_flops);
 
+// ---------------------------------------------------------- adapter merge
+// (nf4_merge.cu) out[n, k] = dequant(W) + scale * B . A, tiles of 128 rows x
+// merge_tile_cols() columns; k_steps = 64-wide steps of the zero-padded rank.
+struct MergeParams {
+  int32_t tiles_m, tiles_n, k_steps;
+  int64_t n, k;
+  const uint8_t* codes;
+  ScaleSrc scales;
+  float scale;
+  void* out;
+  Nf4Table tab;
+};
+struct MergeMaps {
+  CUtensorMap b;       // B [n, r] bf16, box [64, 128], 128B swizzle
+  CUtensorMap a;       // A [r, k] bf16, box [64, 64], 128B swizzle
+  CUtensorMap codes;   // packed codes [n, k/2] u8, box [128, 128], 128B swizzle
+  CUtensorMap out;     // W_out [n, k]: bf16 box [32, 32] 64B swizzle, or fp32 box [32, 32] 128B swizzle
+};
+int merge_tile_cols();
+cudaError_t launch_merge(const MergeParams& p, const MergeMaps& maps, int grid, bool out_f32, cudaStream_t st);
+
 // ------------------------------------------------------------- elementwise
 cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
                                  int32_t r, int32_t r_pad, float scale, float* out_f32,

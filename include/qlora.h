@@ -159,6 +159,27 @@ int qlora_nf4_quantize_noalloc(const float *W, qlora_nf4_weight *w, qlora_stream
 /* Dequantize `w` into out_bf16 ([n, k] bf16, device), bit-exact per the format above. */
 int qlora_nf4_dequantize(const qlora_nf4_weight *w, uint16_t *out_bf16, qlora_stream_t stream);
 
+/*
+ * Merge a trained adapter onto the dequantized weight:
+ *   W_out[n, k] = W'[n, k] + (alpha / r) * (B . A)[n, k]
+ * where W' is the BF16 dequantization of `w` (the format above), A is [r, k]
+ * and B is [n, r] (bf16, row-major, device). A 4-bit matrix cannot absorb
+ * the adapter, so deployment merges it onto a dequantized copy ("QLoRA:
+ * Quantized Low-Rank Adaptation", Price 2: deployment friction; "QLoRA
+ * Explained", Step 5: Save and Merge Adapters). out_dtype QLORA_DTYPE_BF16
+ * stores the BF16 copy; QLORA_DTYPE_FP32 stores fp32 values, ready to be
+ * quantized again with qlora_nf4_quantize for deployment ("QLoRA vs LoRA",
+ * FAQ on converting back to full precision).
+ *  - Each element is fp32(w' + s * acc) with acc the fp32 tensor-core sum of
+ *    the r products, then rounded once more to BF16 for QLORA_DTYPE_BF16.
+ *  - W_out is [n, k] row-major, caller-owned, 16-byte aligned. Requires
+ *    k % 64 == 0 and r in {8, 16, 32, 64, 128}; otherwise
+ *    QLORA_ERR_UNSUPPORTED. Null or misaligned pointers: QLORA_ERR_INVALID.
+ *    Nothing is enqueued on an error. No workspace; nothing is allocated.
+ */
+int qlora_lora_merge(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                     void *W_out, int32_t out_dtype, qlora_stream_t stream);
+
 /* Bytes of device workspace qlora_linear_fwd / qlora_linear_bwd need for m
  * tokens, an [n, k] weight and rank r. */
 size_t qlora_linear_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);

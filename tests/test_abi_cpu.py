@@ -100,6 +100,14 @@ def test_invalid_arguments_rejected_on_host(L):
     rc = L.qlora_linear_bwd(ctypes.byref(ww), 1 << 23, 1 << 24, 128, 1 << 25, 1 << 26, 8, 16.0, None, None, 0,
                             None, 1 << 28, 0, 1 << 29, 1 << 30, None)
     assert rc == 1
+    # adapter merge: null adapter, bad output dtype, unsupported rank or k
+    ww = _weight()
+    assert L.qlora_lora_merge(ctypes.byref(ww), None, 1 << 25, 8, 16.0, 1 << 26, 0, None) == 1
+    assert L.qlora_lora_merge(ctypes.byref(ww), 1 << 24, 1 << 25, 8, 16.0, 1 << 26 | 8, 0, None) == 1
+    assert L.qlora_lora_merge(ctypes.byref(ww), 1 << 24, 1 << 25, 8, 16.0, 1 << 26, 7, None) == 1
+    assert L.qlora_lora_merge(ctypes.byref(ww), 1 << 24, 1 << 25, 12, 16.0, 1 << 26, 0, None) == 2
+    wk = _weight(k=200)
+    assert L.qlora_lora_merge(ctypes.byref(wk), 1 << 24, 1 << 25, 8, 16.0, 1 << 26, 1, None) == 2
     # elementwise
     assert L.qlora_silu_gate_fwd(None, None, None, 16, None) == 1
     assert L.qlora_silu_gate_fwd(None, None, None, 0, None) == 0
