@@ -22,6 +22,7 @@ bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -43,6 +44,27 @@ ALPHA = 16.0
 LAYERS = [("q_proj", 8192, 8192), ("k_proj", 8192, 8192), ("v_proj", 8192, 8192), ("o_proj", 8192, 8192),
           ("gate_proj", 22016, 8192), ("up_proj", 22016, 8192), ("down_proj", 8192, 22016)]
 L2_FLUSH_BYTES = 512 << 20
+
+# DRAM bytes (read + write) per fused-GEMM launch, averaged over the 21 launches of one step, from the
+# 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum; summary in
+# profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
+# recorded with it; any change to them prints null until the counters are taken again.
+WGEMM_TRAFFIC = {"bytes_per_launch": None, "sources_sha256": None}
+WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
+
+
+def wgemm_sources_sha256() -> str:
+    h = hashlib.sha256()
+    for rel in WGEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def wgemm_traffic():
+    if WGEMM_TRAFFIC["sources_sha256"] is None or WGEMM_TRAFFIC["sources_sha256"] != wgemm_sources_sha256():
+        return None
+    return WGEMM_TRAFFIC["bytes_per_launch"]
 
 
 # ------------------------------------------------------------------ helpers --
@@ -532,7 +554,8 @@ def run_native(args) -> None:
     peak_tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
-                "frac": (achieved / peak_tc) if achieved else None, "traffic": None,
+                "frac": (achieved / peak_tc) if achieved else None, "traffic": wgemm_traffic(),
+                "traffic_unit": "DRAM bytes per launch, average over the step's fused-GEMM launches",
                 "kernel": "qlora_wgemm_kernel (fused NF4 dequant + tcgen05, weight as the 128-row operand; forward Y and backward dX)",
                 "launches_timed": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1),
                 "peak_kind": f"bf16_tflops_sustained ({peaks['_source']})"}
