@@ -276,8 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4 codes[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) codes[c] = lds128(crow + (((half * 4 + c) ^ (tr & 7)) << 4));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&code_empty[cs]);
+      const int cs_used = cs;
       if (++cs == kCodeStages) { cs = 0; cph ^= 1; }
 
       if (!mbar_wait(&acc_full[acc], aph)) break;
@@ -311,7 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[acc]);
+        // the code slot is released only after its values were used and the proxy fence above
+        // ordered the reads before the async-proxy refill
+        mbar_arrive(&code_empty[cs_used]);
+      }
       acc ^= 1;
       if (acc == 0) aph ^= 1;
       cur[0] = nxt[0];

@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
       }
       if (kDQ && l == 0) s_tree[lb] = (b < nblk) ? static_cast<double>(m) : 0.0;
     }
+    fence_proxy_async_smem();                 // reads of the stage ordered before its bulk-copy refill
     __syncthreads();                          // stage consumed, tree leaves written
     if (kDQ) {
       // fixed pairwise tree over this chunk's 128 absmax values
@@ -377,6 +378,7 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
         __stcs(dst + (o >> 4), v);
       }
     }
+    fence_proxy_async_smem();                  // reads of the stage ordered before its bulk-copy refill
     __syncthreads();                           // code stage consumed by every warp
     if (tid == 0 && i + kDStages < my_n) issue(i + kDStages);
   }
