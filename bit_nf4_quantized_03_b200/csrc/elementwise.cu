@@ -222,7 +222,7 @@ __global__ void selftest_wait_timeout_kernel(uint64_t limit_ns) {
   fence_mbar_init();
   const uint32_t a = smem_u32(&bar);
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, 0)) {
+  while (!mbar_try_wait_suspend(a, 0, kSuspendHintNs)) {   // the same suspending wait the pipelines use
     if (globaltimer_ns() - t0 > limit_ns) {
       atomicExch(&g_device_error, kErrWaitTimeout);
       return;

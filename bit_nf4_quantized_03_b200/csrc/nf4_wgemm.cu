@@ -485,7 +485,7 @@ int wgemm_bn(int64_t tokens) {
 }
 
 // Ring depths per token-tile width (dequantized tiles, activation tiles, code tiles).
-template <bool kBwd> using WCfg16 = WCfg<16, 8, 8, 16, kBwd>;
+template <bool kBwd> using WCfg16 = WCfg<16, 2, 8, 16, kBwd>;
 template <bool kBwd> using WCfg64 = WCfg<64, 6, 8, 12, kBwd>;
 template <bool kBwd> using WCfg128 = WCfg<128, 4, 6, 12, kBwd>;
 template <bool kBwd> using WCfg256 = WCfg<256, 4, 4, 8, kBwd>;

@@ -177,6 +177,32 @@ Split choose_split(int64_t tiles, int64_t k_tiles, int sms) {
   return s;
 }
 
+// Split of the fused GEMM's reduction over a persistent grid of `sms` CTAs:
+// the split count that minimises the makespan, measured in K steps of one
+// 128-row weight tile (each unit also pays about one step to fill and drain
+// its pipeline), plus the fp32 partial traffic a split adds (written once and
+// read once by the reduction; bytes_per_step converts bytes to K steps).
+Split choose_wsplit(int64_t tiles, int64_t k_tiles, int sms, int64_t out_elems) {
+  const double bytes_per_step = 3.0e6;     // ~0.5 us of one expanded 128 x 64 tile against ~6 TB/s
+  Split best;
+  best.kps = static_cast<int>(std::max<int64_t>(k_tiles, 1));
+  best.splits = 1;
+  double best_cost = 1e300;
+  for (int64_t want = 1; want <= std::min<int64_t>(64, std::max<int64_t>(k_tiles, 1)); ++want) {
+    const int64_t kps = cdiv(std::max<int64_t>(k_tiles, 1), want);
+    const int64_t splits = cdiv(std::max<int64_t>(k_tiles, 1), kps);
+    const int64_t waves = cdiv(tiles * splits, sms);
+    double cost = static_cast<double>(waves) * (static_cast<double>(kps) + 1.0);
+    if (splits > 1) cost += 2.0 * static_cast<double>(splits) * static_cast<double>(out_elems) * 4.0 / bytes_per_step;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best.kps = static_cast<int>(kps);
+      best.splits = static_cast<int>(splits);
+    }
+  }
+  return best;
+}
+
 struct Plan {
   int r_pad = 64;
   GemmKind down_k = kGemmLoraDownK, down_mn = kGemmLoraDownMN, grad = kGemmLoraGrad;
@@ -203,9 +229,9 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   P.bn = wgemm_bn(m);
   const int64_t tok_tiles = cdiv(m, P.bn);
   const int64_t fwd_tiles = cdiv(n, 128) * tok_tiles;
-  if (fwd_tiles * 2 <= sms) P.fwd = choose_split(fwd_tiles, k / 64, sms);
+  P.fwd = choose_wsplit(fwd_tiles, k / 64, sms, m * n);
   const int64_t bwd_tiles = cdiv(k, 128) * tok_tiles;
-  if (bwd_tiles * 2 <= sms) P.bwd = choose_split(bwd_tiles, cdiv(n, 64), sms);
+  P.bwd = choose_wsplit(bwd_tiles, cdiv(n, 64), sms, m * k);
   const size_t rp = static_cast<size_t>(P.r_pad);
   size_t off = 0;
   auto take = [&](size_t bytes) {

@@ -83,19 +83,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (up to `hint_ns`) until the
+// phase completes instead of returning at once, so a waiting warp does not
+// take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete. Gives up after
 // roughly `kWaitLimitNs` of wall time, records kErrWaitTimeout and returns
 // false; every caller then abandons its loop so the whole CTA can exit.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr uint32_t kSuspendHintNs = 20000;         // longest suspension per try (20 us)
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar_ptr, uint32_t parity) {
   const uint32_t bar = smem_u32(bar_ptr);
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
+  uint32_t tries = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 1023u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+    if ((++tries & 15u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
       atomicExch(&g_device_error, kErrWaitTimeout);
       return false;
     }
