@@ -49,7 +49,8 @@ L2_FLUSH_BYTES = 512 << 20
 # 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum; summary in
 # profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
 # recorded with it; any change to them prints null until the counters are taken again.
-WGEMM_TRAFFIC = {"bytes_per_launch": None, "sources_sha256": None}
+WGEMM_TRAFFIC = {"bytes_per_launch": 662939075,
+                 "sources_sha256": "7440c3f92a08ccc2e9a11b4f395b2c0b8ef98f2015abc34d4f3402cbad1f7713"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 
