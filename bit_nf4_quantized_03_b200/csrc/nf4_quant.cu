@@ -75,23 +75,30 @@ __device__ __forceinline__ float absmax8(const float4& a, const float4& b) {
 }
 
 // Fixed pairwise tree (fp64) over part[0..n) zero-padded to a power of two,
-// by one CTA of 256 threads. Each warp reduces an aligned group of 512: every
-// lane sums its 16 consecutive values pairwise, then five xor-shuffle levels
-// combine neighbouring lanes (a + b == b + a exactly, so this is the same
-// tree). Level by level, ping-ponging between `part` and `other`, until one
-// value is left.
-__device__ double tree_sum_cta(double* part, double* other, int64_t n) {
+// by one CTA of 256 threads, without writing global memory (so every CTA of a
+// grid can run it on the same input). Each warp reduces an aligned group of
+// 512: every lane sums its 16 consecutive values pairwise, then five
+// xor-shuffle levels combine neighbouring lanes (a + b == b + a exactly, so
+// this is the same tree). The group sums go to shared memory and the next
+// level runs on them, until one value is left. Zero padding at any level
+// leaves the result unchanged (x + 0 == x), so this equals the tree over the
+// whole power-of-two-padded array. `buf` holds 2 * kTreeBuf doubles.
+constexpr int kTreeBuf = 2048;               // group sums per level: n <= 2048 * 512 on the first level
+
+__device__ double tree_sum_cta(const double* __restrict__ part, int64_t n, double* buf) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  double* src = part;
-  double* dst = other;
+  const double* src = part;
+  bool global_src = true;
+  int pp = 0;
   while (n > 1) {
     const int64_t groups = (n + 511) / 512;
+    double* dst = buf + pp * kTreeBuf;
     for (int64_t g = warp; g < groups; g += 8) {
       double v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int64_t idx = g * 512 + lane * 16 + j;
-        v[j] = (idx < n) ? __ldcg(src + idx) : 0.0;           // other CTAs' sums: read through L2
+        v[j] = (idx < n) ? (global_src ? __ldcg(src + idx) : src[idx]) : 0.0;
       }
 #pragma unroll
       for (int w = 1; w < 16; w <<= 1)
@@ -102,21 +109,15 @@ __device__ double tree_sum_cta(double* part, double* other, int64_t n) {
       for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
       if (lane == 0) dst[g] = t;
     }
-    __threadfence_block();
     __syncthreads();
-    double* sw = src;
     src = dst;
-    dst = sw;
+    global_src = false;
+    pp ^= 1;
     n = groups;
   }
-  return __ldcg(src);
-}
-
-// Mean of all block absmax values from the per-chunk fp64 sums (one CTA).
-__global__ void __launch_bounds__(256) dq_mean_kernel(double* __restrict__ part, double* __restrict__ other,
-                                                      int64_t nchunks, int64_t nblk, float* __restrict__ mean_out) {
-  const double S = tree_sum_cta(part, other, nchunks);
-  if (threadIdx.x == 0) *mean_out = static_cast<float>(S / static_cast<double>(nblk));
+  const double r = global_src ? __ldcg(src) : src[0];
+  __syncthreads();
+  return r;
 }
 
 template <bool kDQ>
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
                                                               double* __restrict__ part_out) {
   extern __shared__ __align__(128) uint8_t q_stage[];
   __shared__ float2 s_tab[64];
-  __shared__ double s_tree[kQChunk];
+  __shared__ double s_part[2][kQChunk / 4];   // per chunk: sums of 4 adjacent blocks (double-buffered by chunk)
   __shared__ __align__(8) uint64_t full[kQStages];
   const int tid = threadIdx.x;
   const int grp = tid >> 3;          // one 64-block per group of eight lanes
@@ -228,57 +229,76 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
         if (kDQ) absmax_out[b] = m;
         else scale_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
       }
-      if (kDQ && l == 0) s_tree[lb] = (b < nblk) ? static_cast<double>(m) : 0.0;
+      if (kDQ) {
+        // first two levels of the fixed pairwise tree: the warp's four groups hold four
+        // adjacent blocks (lb = it*32 + 4*warp + 0..3), all eight lanes of a group hold its m
+        double t = (b < nblk) ? static_cast<double>(m) : 0.0;
+        t = t + __shfl_xor_sync(0xffffffffu, t, 8);
+        t = t + __shfl_xor_sync(0xffffffffu, t, 16);
+        if ((tid & 31) == 0) s_part[i & 1][it * 8 + (tid >> 5)] = t;
+      }
     }
     fence_proxy_async_smem();                 // reads of the stage ordered before its bulk-copy refill
-    __syncthreads();                          // stage consumed, tree leaves written
-    if (kDQ) {
-      // fixed pairwise tree over this chunk's 128 absmax values
-      double t = 0.0;
-      if (tid < kQChunk / 2) t = s_tree[2 * tid] + s_tree[2 * tid + 1];
-      __syncthreads();
-      if (tid < kQChunk / 2) s_tree[tid] = t;
-      __syncthreads();
-      for (int stride = 1; stride < kQChunk / 2; stride <<= 1) {
-        if (tid < kQChunk / 2 && (tid & (2 * stride - 1)) == 0) s_tree[tid] = s_tree[tid] + s_tree[tid + stride];
-        __syncthreads();
-      }
-      if (tid == 0) part_out[blockIdx.x + i * gridDim.x] = s_tree[0];
-      __syncthreads();
+    __syncthreads();                          // stage consumed, tree nodes written
+    if (kDQ && tid < 32) {
+      // remaining five levels over the chunk's 32 nodes, in index order (xor-shuffle pairs)
+      double t = s_part[i & 1][tid];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
+      if (tid == 0) part_out[blockIdx.x + i * gridDim.x] = t;
     }
     if (tid == 0 && i + kQStages < my_n) issue(i + kQStages);
   }
 }
 
 // ---------------------------------------------------------------------------
-// Stage 2: per 256-block, d = a - mean, s2 = max|d| / 448, q = e4m3(d / s2).
-// One CTA of 256 threads per second-level block.
+// Stage 2: the mean, then per 256-block d = a - mean, s2 = max|d| / 448,
+// q = e4m3(d / s2). Every CTA sums the per-chunk partials with the same fixed
+// tree (bit-identical results, no extra launch for the mean). Its up to
+// kFinishPer 256-blocks (one absmax per thread each) are requested before the
+// tree so the loads overlap it, and all of them are reduced in one barrier.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) dq_fp8_kernel(const float* __restrict__ absmax, int64_t nblk,
-                                                      const float* __restrict__ mean_in,
-                                                      uint8_t* __restrict__ q_out,
-                                                      float* __restrict__ s2_out,
-                                                      float* __restrict__ mean_out) {
-  __shared__ float wmax[8];
-  const float mean = *mean_in;
-  const int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
-  const bool valid = b < nblk;
-  const float d = valid ? __fsub_rn(absmax[b], mean) : 0.f;
-  float m = fabsf(d);
+constexpr int kFinishPer = 8;                 // 256-blocks per CTA, loaded up front
+
+__global__ void __launch_bounds__(256) dq_finish_kernel(const double* __restrict__ part, int64_t nchunks,
+                                                         const float* __restrict__ absmax, int64_t nblk,
+                                                         uint8_t* __restrict__ q_out, float* __restrict__ s2_out,
+                                                         float* __restrict__ mean_out) {
+  __shared__ double tree_buf[2 * kTreeBuf];
+  __shared__ float wmax[kFinishPer][8];
+  const int64_t nb2 = (nblk + 255) / 256;
+  // this CTA's absmax values, requested before the mean so the loads overlap the tree
+  float a[kFinishPer];
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-  __syncthreads();
-  float amax = wmax[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, wmax[i]);
-  const float s2 = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-  if (valid) {
-    q_out[b] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(d, s2), __NV_SATFINITE, __NV_E4M3));
+  for (int j = 0; j < kFinishPer; ++j) {
+    const int64_t b = (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(j) * gridDim.x) * 256 + threadIdx.x;
+    a[j] = (b < nblk) ? __ldcg(absmax + b) : 0.f;
   }
-  if (threadIdx.x == 0) {
-    s2_out[blockIdx.x] = s2;
-    if (blockIdx.x == 0) *mean_out = mean;
+  const double S = tree_sum_cta(part, nchunks, tree_buf);
+  const float mean = static_cast<float>(S / static_cast<double>(nblk));
+  if (blockIdx.x == 0 && threadIdx.x == 0) *mean_out = mean;
+  float d[kFinishPer];
+#pragma unroll
+  for (int j = 0; j < kFinishPer; ++j) {
+    const int64_t b = (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(j) * gridDim.x) * 256 + threadIdx.x;
+    d[j] = (b < nblk) ? __fsub_rn(a[j], mean) : 0.f;
+    float m = fabsf(d[j]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) wmax[j][threadIdx.x >> 5] = m;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kFinishPer; ++j) {
+    const int64_t c = static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(j) * gridDim.x;
+    if (c >= nb2) break;
+    float amax = wmax[j][0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, wmax[j][i]);
+    const float s2 = (amax == 0.f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+    const int64_t b = c * 256 + threadIdx.x;
+    if (b < nblk) q_out[b] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(d[j], s2), __NV_SATFINITE, __NV_E4M3));
+    if (threadIdx.x == 0) s2_out[c] = s2;
   }
 }
 
@@ -433,8 +453,6 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   const QuantWsLayout L = quant_ws_layout(n_elem);
   float* absmax = reinterpret_cast<float*>(static_cast<char*>(ws) + L.absmax_off);
   double* part_a = reinterpret_cast<double*>(static_cast<char*>(ws) + L.part_a_off);
-  double* part_b = reinterpret_cast<double*>(static_cast<char*>(ws) + L.part_b_off);
-  float* mean_tmp = reinterpret_cast<float*>(static_cast<char*>(ws) + L.mean_off);
   // stage 1 also writes one fp64 tree sum per chunk (the first levels of the fixed-order sum)
   e = set_smem_once(nf4_quantize_kernel<true>, kQSmem, smem_set[1]);
   if (e != cudaSuccess) return e;
@@ -442,13 +460,13 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // the rest of the tree and the mean
-  dq_mean_kernel<<<1, 256, 0, st>>>(part_a, part_b, nchunks, nblk, mean_tmp);
-  count_launches(1);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  // the rest of the tree, the mean and the E4M3 pass in one launch
   const int64_t nb2 = (nblk + 255) / 256;
-  dq_fp8_kernel<<<static_cast<int>(nb2), 256, 0, st>>>(absmax, nblk, mean_tmp, scale_fp8, dq_scale, dq_mean);
+  // enough CTAs that each takes at most kFinishPer 256-blocks, at least one per SM when there is work
+  int64_t g2 = (nb2 + kFinishPer - 1) / kFinishPer;
+  if (g2 < num_sms) g2 = nb2 < num_sms ? nb2 : num_sms;
+  const int grid2 = static_cast<int>(g2);
+  dq_finish_kernel<<<grid2, 256, 0, st>>>(part_a, nchunks, absmax, nblk, scale_fp8, dq_scale, dq_mean);
   count_launches(1);
   return cudaGetLastError();
 }

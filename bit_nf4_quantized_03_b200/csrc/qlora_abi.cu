@@ -384,6 +384,7 @@ int qlora_nf4_quantize(const float* W, qlora_nf4_weight* w, void* ws, size_t ws_
   const int64_t n_elem = w->n * w->k;
   const bool dq = (w->mode == QLORA_SCALE_DQ_FP8);
   if (dq) {
+    if (n_elem > kMaxDqElems) return QLORA_ERR_UNSUPPORTED;
     if (ws == nullptr || !aligned16(ws) || ws_bytes < quant_ws_layout(n_elem).total) return QLORA_ERR_WORKSPACE;
   }
   const cudaError_t e =

@@ -29,6 +29,10 @@ inline QuantWsLayout quant_ws_layout(int64_t n_elem) {
   return L;
 }
 
+// Largest tensor the double-quant mean supports: the fixed tree keeps at most 2048
+// first-level group sums (groups of 512 chunk partials of 128 blocks of 64 weights).
+constexpr int64_t kMaxDqElems = int64_t(2048) * 512 * 128 * 64;
+
 cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab, const Nf4Buckets& bk,
                             uint8_t* codes, uint16_t* scale_bf16, uint8_t* scale_fp8, float* dq_scale,
                             float* dq_mean, void* ws, int num_sms, cudaStream_t st);

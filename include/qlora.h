@@ -130,7 +130,8 @@ size_t qlora_nf4_quantize_workspace_bytes(int64_t n, int64_t k, int32_t mode);
 /*
  * Quantize W (fp32 [n, k], device) into `w` (buffers and shape set by the
  * caller). Any n*k >= 1 (the last block may be partial). The double-quant
- * mode needs `ws` of at least qlora_nf4_quantize_workspace_bytes bytes.
+ * mode needs `ws` of at least qlora_nf4_quantize_workspace_bytes bytes and
+ * n*k <= 2^33 (QLORA_ERR_UNSUPPORTED above that, nothing enqueued).
  * Deterministic: the same input gives the same bytes on every call.
  */
 int qlora_nf4_quantize(const float *W, qlora_nf4_weight *w, void *ws, size_t ws_bytes, qlora_stream_t stream);
