@@ -59,6 +59,18 @@ design notes of the repository):
    for deployment): W_merged = W' + (alpha/r) B A, exact in fp64 here; the
    stored BF16 or FP32 copy is that value rounded once (checked by the
    tests with the bound their docstrings derive).
+10. LoRA dropout ([GAMUT] Step 3, LoraConfig lora_dropout=0.05, and the
+   hyperparameter quick reference; the pages give only the rate): inverted
+   dropout on the input of the low-rank branch, as PEFT applies it. With a
+   keep mask M and keep scale c = 1/(1 - p): Y = X W'^T + s (c (M*X) A^T) B^T;
+   dA = s c (dY B)^T (M*X); dX = dY W' + s c ((dY B) A) * M; dB = s dY^T U
+   with U = c (M*X) A^T. The mask is drawn from Philox4x32-10 (Salmon et al.,
+   "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011), counter =
+   (e // 8 as two 32-bit words, offset as two 32-bit words), key = seed as
+   two 32-bit words; element e (row-major index into X) takes 16-bit lane
+   e % 8 of the four output words (word (e % 8) // 2, low half first) and is
+   kept iff that value >= round(p * 65536). The effective drop rate is
+   round(p * 65536) / 65536 and c = 65536 / (65536 - round(p * 65536)).
 """
 from __future__ import annotations
 
@@ -354,6 +366,99 @@ def lora_merge(Wd, A, B, alpha: float) -> np.ndarray:
     Wd, A, B = _f64(Wd), _f64(A), _f64(B)
     s = float(alpha) / A.shape[0]
     return Wd + s * (B @ A)
+
+
+# ----------------------------------------------------------------------------
+# LoRA dropout (reading 10): Philox4x32-10 keep mask and the dropped layer
+# ----------------------------------------------------------------------------
+PHILOX_M0, PHILOX_M1 = 0xD2511F53, 0xCD9E8D57      # round multipliers
+PHILOX_W0, PHILOX_W1 = 0x9E3779B9, 0xBB67AE85      # key increments (Weyl sequence)
+M32 = 0xFFFFFFFF
+
+
+def philox4x32_10(c0, c1, c2, c3, k0, k1):
+    """Philox4x32 with 10 rounds on uint64 numpy arrays holding 32-bit values:
+    each round multiplies c0 and c2 by the two constants (64-bit products split
+    into high and low words) and mixes the high words with c1, c3 and the key;
+    the key advances by the Weyl increments between rounds."""
+    c0, c1, c2, c3 = (np.asarray(v, dtype=np.uint64) & M32 for v in (c0, c1, c2, c3))
+    k0 = np.asarray(k0, dtype=np.uint64) & M32
+    k1 = np.asarray(k1, dtype=np.uint64) & M32
+    for rnd in range(10):
+        p0 = c0 * np.uint64(PHILOX_M0)
+        p1 = c2 * np.uint64(PHILOX_M1)
+        hi0, lo0 = p0 >> np.uint64(32), p0 & np.uint64(M32)
+        hi1, lo1 = p1 >> np.uint64(32), p1 & np.uint64(M32)
+        c0, c1, c2, c3 = hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0
+        if rnd < 9:
+            k0 = (k0 + np.uint64(PHILOX_W0)) & np.uint64(M32)
+            k1 = (k1 + np.uint64(PHILOX_W1)) & np.uint64(M32)
+    return c0, c1, c2, c3
+
+
+def dropout_threshold(p: float) -> int:
+    """16-bit drop threshold round(p * 65536); p must lie in [0, 1)."""
+    t = int(round(float(p) * 65536.0))
+    if not 0 <= t < 65536:
+        raise ValueError("dropout rate must lie in [0, 1)")
+    return t
+
+
+def dropout_keep_scale(p: float) -> float:
+    t = dropout_threshold(p)
+    return 65536.0 / (65536.0 - t)
+
+
+def dropout_random16(count: int, seed: int, offset: int) -> np.ndarray:
+    """The 16-bit random value of each element e in [0, count)."""
+    e = np.arange(count, dtype=np.uint64)
+    g = e >> np.uint64(3)
+    words = philox4x32_10(g & np.uint64(M32), g >> np.uint64(32), offset & M32, (offset >> 32) & M32,
+                          seed & M32, (seed >> 32) & M32)
+    lane = (e & np.uint64(7)).astype(np.int64)
+    w = np.choose(lane >> 1, words)
+    return ((w >> ((lane & 1) * 16).astype(np.uint64)) & np.uint64(0xFFFF)).astype(np.uint32)
+
+
+def dropout_mask(m: int, k: int, p: float, seed: int, offset: int) -> np.ndarray:
+    """Boolean keep mask [m, k] of reading 10."""
+    return (dropout_random16(m * k, seed, offset) >= dropout_threshold(p)).reshape(m, k)
+
+
+def pack_mask_bits(mask) -> np.ndarray:
+    """Row-major bit packing: element e -> bit e % 8 of byte e // 8."""
+    return np.packbits(np.asarray(mask, dtype=np.uint8).reshape(-1), bitorder="little")
+
+
+def linear_forward_dropout(Wd, X, A, B, alpha: float, mask, p: float, rows=None):
+    """Y and U of the layer with dropout on the low-rank input (reading 10)."""
+    c = dropout_keep_scale(p)
+    Wd, X, A, B = _f64(Wd), _f64(X), _f64(A), _f64(B)
+    Xm = X * np.asarray(mask, dtype=np.float64)
+    if rows is not None:
+        X, Xm = X[np.asarray(rows)], Xm[np.asarray(rows)]
+    s = float(alpha) / A.shape[0]
+    U = c * (Xm @ A.T)
+    return X @ Wd.T + s * (U @ B.T), U
+
+
+def linear_backward_dropout(Wd, X, dY, A, B, alpha: float, mask, p: float, dx_rows=None):
+    """dX, dA, dB of the layer with dropout on the low-rank input (reading 10)."""
+    c = dropout_keep_scale(p)
+    Wd, X, dY, A, B = _f64(Wd), _f64(X), _f64(dY), _f64(A), _f64(B)
+    Mf = np.asarray(mask, dtype=np.float64)
+    Xm = X * Mf
+    s = float(alpha) / A.shape[0]
+    G = dY @ B
+    U = c * (Xm @ A.T)
+    dB = s * (dY.T @ U)
+    dA = s * c * (G.T @ Xm)
+    if dx_rows is not None:
+        r_ = np.asarray(dx_rows)
+        dX = dY[r_] @ Wd + s * c * ((G[r_] @ A) * Mf[r_])
+    else:
+        dX = dY @ Wd + s * c * ((G @ A) * Mf)
+    return dX, dA, dB
 
 
 def silu_gate_forward(g, u):

@@ -410,3 +410,91 @@ def test_lora_merge_against_python_loops_and_the_layer():
     # the update has rank at most r
     sv = np.linalg.svd(Wm - Wd, compute_uv=False)
     assert np.all(sv[3:] <= 1e-12 * sv[0])
+
+
+# ---------------------------------------------------------------- LoRA dropout
+def test_dropout_keep_rate_and_uniformity():
+    # reading 10: 16-bit values uniform on [0, 65536); kept iff >= round(p * 65536)
+    n = 1 << 22
+    r = o.dropout_random16(n, seed=20231, offset=5)
+    assert r.min() >= 0 and r.max() <= 0xFFFF
+    hist = np.bincount((r >> 8).astype(np.int64), minlength=256)
+    expect = n / 256.0
+    chi2 = float(np.sum((hist - expect) ** 2 / expect))
+    assert chi2 < 255 + 6 * np.sqrt(2 * 255), chi2            # 255 dof, ~6 sigma
+    for lane in range(8):                                       # every 16-bit lane of the 4 words is used alike
+        mu = r[lane::8].mean()
+        assert abs(mu - 32767.5) < 6 * 18918.0 / np.sqrt(n / 8), (lane, mu)
+    p = 0.05
+    keep = (r >= o.dropout_threshold(p)).mean()
+    q = o.dropout_threshold(p) / 65536.0
+    assert abs(keep - (1 - q)) < 6 * np.sqrt(q * (1 - q) / n), keep
+    assert o.dropout_threshold(p) == 3277 and abs(o.dropout_keep_scale(p) - 65536 / 62259) < 1e-15
+
+
+def test_dropout_streams_are_independent():
+    m, k, p = 512, 1024, 0.05
+    a = o.dropout_mask(m, k, p, seed=1, offset=0)
+    for other in (o.dropout_mask(m, k, p, seed=2, offset=0), o.dropout_mask(m, k, p, seed=1, offset=1)):
+        diff = np.mean(a != other)
+        q = o.dropout_threshold(p) / 65536.0
+        assert abs(diff - 2 * q * (1 - q)) < 0.01, diff           # independent masks disagree at rate 2q(1-q)
+    # neighbouring elements (same Philox call, and across calls) are uncorrelated
+    x = a.reshape(-1).astype(np.float64)
+    for lag in (1, 2, 7, 8, 9):
+        c = np.corrcoef(x[:-lag], x[lag:])[0, 1]
+        assert abs(c) < 0.01, (lag, c)
+    assert np.array_equal(a, o.dropout_mask(m, k, p, seed=1, offset=0))   # deterministic in (seed, offset)
+
+
+def test_dropout_zero_rate_is_the_plain_layer():
+    Wd, X, A, B, dY = _tiny_layer(M=5, N=6, K=128, r=4)
+    mask = o.dropout_mask(5, 128, 0.0, seed=3, offset=0)
+    assert mask.all() and o.dropout_keep_scale(0.0) == 1.0
+    Y, U = o.linear_forward(Wd, X, A, B, 16.0)
+    Yd, Ud = o.linear_forward_dropout(Wd, X, A, B, 16.0, mask, 0.0)
+    assert np.array_equal(Y, Yd) and np.array_equal(U, Ud)
+    g = o.linear_backward(Wd, X, dY, A, B, 16.0)
+    gd = o.linear_backward_dropout(Wd, X, dY, A, B, 16.0, mask, 0.0)
+    for a, b in zip(g, gd):
+        np.testing.assert_allclose(a, b, rtol=1e-14, atol=1e-15)
+
+
+def test_dropout_layer_against_loops_and_finite_differences():
+    Wd, X, A, B, dY = _tiny_layer(M=4, N=6, K=64, r=2)
+    p = 0.3
+    mask = o.dropout_mask(4, 64, p, seed=11, offset=2)
+    assert 0 < mask.mean() < 1
+    c = 65536.0 / (65536.0 - round(p * 65536))
+    Y, _ = o.linear_forward_dropout(Wd, X, A, B, 16.0, mask, p)
+    s = 16.0 / 2
+    for i in range(4):                                            # Python loops over the definition
+        for j in range(6):
+            base = sum(float(X[i, t]) * float(Wd[j, t]) for t in range(64))
+            low = 0.0
+            for q in range(2):
+                u = c * sum(float(X[i, t]) * float(mask[i, t]) * float(A[q, t]) for t in range(64))
+                low += u * float(B[j, q])
+            assert abs(Y[i, j] - (base + s * low)) < 1e-12 * (1 + abs(Y[i, j]))
+
+    def loss(Xv, Av, Bv):
+        return float(np.sum(o.linear_forward_dropout(Wd, Xv, Av, Bv, 16.0, mask, p)[0] * dY))
+
+    dX, dA, dB = o.linear_backward_dropout(Wd, X, dY, A, B, 16.0, mask, p)
+    h = 1e-4
+    for name, T, G in (("X", X, dX), ("A", A, dA), ("B", B, dB)):
+        num = np.zeros_like(T)
+        for idx in np.ndindex(T.shape):
+            Tp, Tm = T.copy(), T.copy()
+            Tp[idx] += h
+            Tm[idx] -= h
+            args_p = {"X": (Tp, A, B), "A": (X, Tp, B), "B": (X, A, Tp)}[name]
+            args_m = {"X": (Tm, A, B), "A": (X, Tm, B), "B": (X, A, Tm)}[name]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(G, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_mask_bit_packing_order():
+    mask = np.zeros((2, 16), dtype=bool)
+    mask[0, 0] = mask[0, 9] = mask[1, 15] = True
+    assert o.pack_mask_bits(mask).tolist() == [0x01, 0x02, 0x00, 0x80]
