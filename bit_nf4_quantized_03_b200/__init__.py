@@ -35,6 +35,7 @@ EXPORTED = (
     "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_check_device_error",
     "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end",
     "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
+    "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
 )
 
 
@@ -56,6 +57,20 @@ class NF4Weight(ctypes.Structure):
     ]
 
 
+class Dropout(ctypes.Structure):
+    """Mirror of qlora_dropout: LoRA dropout rate, Philox seed and offset, and the
+    device mask buffer (m * k / 8 bytes) the forward writes and the backward reads."""
+    _fields_ = [
+        ("p", ctypes.c_float), ("reserved", ctypes.c_int32),
+        ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64),
+        ("mask", ctypes.c_void_p),
+    ]
+
+    def __init__(self, p: float, seed: int, offset: int, mask):
+        super().__init__(float(p), 0, int(seed), int(offset), _ptr(mask))
+        self._mask = mask
+
+
 _lib = None
 
 
@@ -69,6 +84,7 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
     pw = ctypes.POINTER(NF4Weight)
+    pd = ctypes.POINTER(Dropout)
     sig = {
         "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "qlora_version": (ctypes.c_char_p, []),
@@ -89,6 +105,10 @@ def lib() -> ctypes.CDLL:
         "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
         "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
+        "qlora_linear_workspace_bytes_ex": (sz, [i64, i64, i64, i32, pd]),
+        "qlora_linear_fwd_ex": (ctypes.c_int, [pw, vp, i64, vp, vp, i32, f32, vp, i32, vp, pd, vp, sz, vp]),
+        "qlora_linear_bwd_ex": (ctypes.c_int, [pw, vp, vp, i64, vp, vp, i32, f32, vp, vp, i32, vp, vp, i32,
+                                               pd, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -217,6 +237,34 @@ def qlora_linear_bwd(w: QuantizedWeight, X, dY, A, B, r: int, alpha: float, U_sa
                                 _ptr(dX), dx_dtype, _ptr(dA), _ptr(dB), flags, _ptr(ws), ws_bytes,
                                 _stream(stream))
     _check(rc, "qlora_linear_bwd")
+
+
+def _dref(drop):
+    return None if drop is None else ctypes.byref(drop)
+
+
+def qlora_linear_workspace_bytes_ex(m: int, n: int, k: int, r: int, drop=None) -> int:
+    return int(lib().qlora_linear_workspace_bytes_ex(m, n, k, r, _dref(drop)))
+
+
+def qlora_linear_fwd_ex(w: QuantizedWeight, X, A, B, r: int, alpha: float, Y, y_dtype: int,
+                        U_save=None, drop=None, ws=None, stream=None):
+    m = X.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().qlora_linear_fwd_ex(w.ref(), _ptr(X), m, _ptr(A), _ptr(B), r, float(alpha), _ptr(Y), y_dtype,
+                                   _ptr(U_save), _dref(drop), _ptr(ws), ws_bytes, _stream(stream))
+    _check(rc, "qlora_linear_fwd_ex")
+    return Y
+
+
+def qlora_linear_bwd_ex(w: QuantizedWeight, X, dY, A, B, r: int, alpha: float, U_saved, dX, dx_dtype: int,
+                        dA, dB, flags: int = 0, drop=None, ws=None, stream=None):
+    m = X.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().qlora_linear_bwd_ex(w.ref(), _ptr(X), _ptr(dY), m, _ptr(A), _ptr(B), r, float(alpha),
+                                   _ptr(U_saved), _ptr(dX), dx_dtype, _ptr(dA), _ptr(dB), flags, _dref(drop),
+                                   _ptr(ws), ws_bytes, _stream(stream))
+    _check(rc, "qlora_linear_bwd_ex")
 
 
 def qlora_silu_gate_fwd(g, u, h, stream=None):

@@ -19,7 +19,7 @@ static int blocks_for(int64_t n, int threads) {
 __global__ void lora_finalize_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
                                      int r, int r_pad, float scale, float* __restrict__ out_f32,
                                      uint16_t* __restrict__ out_scaled, uint16_t* __restrict__ out_hi,
-                                     uint16_t* __restrict__ out_lo) {
+                                     uint16_t* __restrict__ out_lo, float pre) {
   const int64_t total = rows * r_pad;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -28,6 +28,7 @@ __global__ void lora_finalize_kernel(const float* __restrict__ part, int splits,
     float s = 0.f;
     if (j < r)
       for (int t = 0; t < splits; ++t) s += part[t * part_stride + idx];
+    s = __fmul_rn(pre, s);
     if (out_f32 != nullptr && j < r) out_f32[row * r + j] = s;
     if (out_scaled != nullptr) out_scaled[idx] = f2bf(__fmul_rn(scale, s));
     if (out_hi != nullptr) {
@@ -40,10 +41,10 @@ __global__ void lora_finalize_kernel(const float* __restrict__ part, int splits,
 
 cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows, int32_t r,
                                  int32_t r_pad, float scale, float* out_f32, uint16_t* out_scaled_bf16,
-                                 uint16_t* out_hi, uint16_t* out_lo, cudaStream_t st) {
+                                 uint16_t* out_hi, uint16_t* out_lo, cudaStream_t st, float pre) {
   const int64_t total = rows * r_pad;
   lora_finalize_kernel<<<blocks_for(total, 256), 256, 0, st>>>(part, splits, part_stride, rows, r, r_pad, scale,
-                                                                out_f32, out_scaled_bf16, out_hi, out_lo);
+                                                                out_f32, out_scaled_bf16, out_hi, out_lo, pre);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -198,7 +199,7 @@ int lora_down_small_slices(int64_t k) { return static_cast<int>((k + kSmallSlice
 
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
                                    int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, float pre) {
   const int ks = lora_down_small_slices(k);
   const dim3 grid(static_cast<unsigned>(r), static_cast<unsigned>(ks));
   if (m <= 16)
@@ -208,7 +209,7 @@ cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, cons
   count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_lora_finalize(part, ks, m * r_pad, m, r, r_pad, scale, U32, sU, nullptr, nullptr, st);
+  return launch_lora_finalize(part, ks, m * r_pad, m, r, r_pad, scale, U32, sU, nullptr, nullptr, st, pre);
 }
 
 // ---------------------------------------------------------------------------

@@ -82,6 +82,47 @@ __device__ __forceinline__ void store_row32(const GemmParams& p, int split, int 
     return;
   }
   const bool full = (col0 + 32 <= p.cols);
+  if (p.out_mode == kOutMaskAccBF16 || p.out_mode == kOutMaskAccF32) {
+    // dropout dX: out += keep_scale * D where the mask keeps the element (the 32 columns start on a
+    // multiple of 32 of a row whose length is a multiple of 64, so their bits are one aligned word)
+    const int64_t e0 = static_cast<int64_t>(row) * p.ld_out + col0;
+    const uint32_t bits = __ldg(reinterpret_cast<const uint32_t*>(p.mask + e0 / 8));
+    if (p.out_mode == kOutMaskAccF32) {
+      float* o = static_cast<float*>(p.out) + e0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 y = *reinterpret_cast<const float4*>(o + j);
+        y.x += ((bits >> j) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j])) : 0.f;
+        y.y += ((bits >> (j + 1)) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j + 1])) : 0.f;
+        y.z += ((bits >> (j + 2)) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j + 2])) : 0.f;
+        y.w += ((bits >> (j + 3)) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j + 3])) : 0.f;
+        *reinterpret_cast<float4*>(o + j) = y;
+      }
+    } else {
+      uint16_t* o = static_cast<uint16_t*>(p.out) + e0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        const uint4 y = *reinterpret_cast<const uint4*>(o + j);
+        const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
+        float x[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          x[2 * t] = __uint_as_float(yy[t] << 16);
+          x[2 * t + 1] = __uint_as_float(yy[t] & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          if ((bits >> (j + t)) & 1u) x[t] += __fmul_rn(p.keep_scale, __uint_as_float(v[j + t]));
+        uint4 w;
+        w.x = pack_bf16x2(x[0], x[1]);
+        w.y = pack_bf16x2(x[2], x[3]);
+        w.z = pack_bf16x2(x[4], x[5]);
+        w.w = pack_bf16x2(x[6], x[7]);
+        *reinterpret_cast<uint4*>(o + j) = w;
+      }
+    }
+    return;
+  }
   if (p.out_mode == kOutF32) {
     float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.ld_out + col0;
     if (full) {

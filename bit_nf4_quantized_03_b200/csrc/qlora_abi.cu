@@ -304,7 +304,7 @@ bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint
 // Low-rank product U (or G): partial GEMM over the reduction, then finalize.
 int run_lora_down(const Plan& P, bool b_mn, const uint16_t* act, int64_t m, int64_t red, const uint16_t* adapter,
                   int32_t r, float scale, char* ws, float* out_f32, uint16_t* out_scaled, uint16_t* out_hi,
-                  uint16_t* out_lo, cudaStream_t st) {
+                  uint16_t* out_lo, cudaStream_t st, float pre = 1.0f) {
   const Split sp = b_mn ? P.g : P.u;
   GemmParams p = base_params(m, P.r_pad, P.r_pad, b_mn ? cdiv(red, 64) : red / 64, sp);
   p.out = ws + P.off_part;
@@ -323,8 +323,58 @@ int run_lora_down(const Plan& P, bool b_mn, const uint16_t* act, int64_t m, int6
   cudaError_t e = launch_gemm(b_mn ? P.down_mn : P.down_k, p, maps, grid_of(p), st);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   e = launch_lora_finalize(static_cast<const float*>(p.out), sp.splits, p.part_stride, m, r, P.r_pad, scale,
-                           out_f32, out_scaled, out_hi, out_lo, st);
+                           out_f32, out_scaled, out_hi, out_lo, st, pre);
   return cuda_status(e);
+}
+
+// Dropout settings resolved on the host: 16-bit threshold and keep scale c.
+struct Drop {
+  bool on = false;
+  uint32_t thr = 0;
+  float keep = 1.0f;
+  uint64_t seed = 0, offset = 0;
+  uint8_t* mask = nullptr;
+};
+
+// QLORA_OK, or QLORA_ERR_INVALID for a rate outside [0, 1) or a missing/misaligned mask.
+int resolve_drop(const qlora_dropout* d, Drop* out) {
+  *out = Drop{};
+  if (d == nullptr || d->p == 0.0f) return QLORA_OK;
+  if (!(d->p > 0.0f && d->p < 1.0f)) return QLORA_ERR_INVALID;
+  const double t = std::nearbyint(static_cast<double>(d->p) * 65536.0);
+  if (t >= 65536.0) return QLORA_ERR_INVALID;
+  if (d->mask == nullptr || !aligned16(d->mask)) return QLORA_ERR_INVALID;
+  out->thr = static_cast<uint32_t>(t);
+  if (out->thr == 0) return QLORA_OK;                     // rounds to no dropout
+  out->on = true;
+  out->keep = static_cast<float>(65536.0 / (65536.0 - t));
+  out->seed = d->seed;
+  out->offset = d->offset;
+  out->mask = d->mask;
+  return QLORA_OK;
+}
+
+size_t drop_ws_bytes(int64_t m, int64_t k) { return align_up(static_cast<size_t>(m) * k * 2, 256); }
+
+// dX += keep * M * ((sG) A): the low-rank term of dX under dropout, one tcgen05 GEMM over the
+// rank with the mask applied in the epilogue.
+int run_lora_up_masked(const Plan& P, const uint16_t* sG, int64_t m, int64_t k, const uint16_t* A, int32_t r,
+                       const Drop& D, void* dX, bool dx_f32, cudaStream_t st) {
+  Split sp;
+  sp.splits = 1;
+  sp.kps = P.r_pad / 64;
+  GemmParams p = base_params(m, k, gemm_bn(P.down_mn), P.r_pad / 64, sp);
+  p.out = dX;
+  p.ld_out = k;
+  p.out_mode = dx_f32 ? kOutMaskAccF32 : kOutMaskAccBF16;
+  p.mask = D.mask;
+  p.keep_scale = D.keep;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  bool ok = map_bf16(&maps.a, sG, m, P.r_pad, 128);                              // [m, r_pad], K-major
+  ok = ok && tmap_2d(&maps.b, A, kBF16, k, r, k * 2, 64, 64, 128);                 // A [r, k]: MN-major
+  if (!ok) return QLORA_ERR_CUDA;
+  return cuda_status(launch_gemm(P.down_mn, p, maps, grid_of(p), st));
 }
 
 // dB (rows = n, act = dY) or dA^T (rows = k, act = X): sum over tokens of act^T . [hi + lo].
@@ -406,6 +456,13 @@ size_t qlora_linear_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r) 
   return make_plan(m, n, k, r).total;
 }
 
+size_t qlora_linear_workspace_bytes_ex(int64_t m, int64_t n, int64_t k, int32_t r, const qlora_dropout* drop) {
+  const size_t base = qlora_linear_workspace_bytes(m, n, k, r);
+  Drop D;
+  if (base == 0 || resolve_drop(drop, &D) != QLORA_OK) return 0;
+  return base + (D.on ? drop_ws_bytes(m, k) : 0);
+}
+
 int qlora_lora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int32_t r, float alpha,
                      void* W_out, int32_t out_dtype, qlora_stream_t stream) {
   if (!weight_ok(w) || A == nullptr || B == nullptr || W_out == nullptr) return QLORA_ERR_INVALID;
@@ -443,26 +500,43 @@ int qlora_lora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_
 int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, const uint16_t* A, const uint16_t* B,
                      int32_t r, float alpha, void* Y, int32_t y_dtype, float* U_save, void* ws, size_t ws_bytes,
                      qlora_stream_t stream) {
+  return qlora_linear_fwd_ex(w, X, m, A, B, r, alpha, Y, y_dtype, U_save, nullptr, ws, ws_bytes, stream);
+}
+
+int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, const uint16_t* A,
+                        const uint16_t* B, int32_t r, float alpha, void* Y, int32_t y_dtype, float* U_save,
+                        const qlora_dropout* drop, void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (!linear_args_ok(w, X, m, A, B, r) || Y == nullptr || !aligned16(Y)) return QLORA_ERR_INVALID;
   if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_FP32) return QLORA_ERR_INVALID;
   if (U_save != nullptr && !aligned16(U_save)) return QLORA_ERR_INVALID;
   const int sst = linear_shape_status(w, r);
   if (sst != QLORA_OK) return sst;
+  Drop D;
+  if (resolve_drop(drop, &D) != QLORA_OK) return QLORA_ERR_INVALID;
   const int64_t n = w->n, k = w->k;
   const Plan P = make_plan(m, n, k, r);
-  if (ws == nullptr || !aligned16(ws) || ws_bytes < P.total) return QLORA_ERR_WORKSPACE;
+  const size_t need = P.total + (D.on ? drop_ws_bytes(m, k) : 0);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < need) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* wsb = static_cast<char*>(ws);
   const float s = alpha / static_cast<float>(r);
   uint16_t* sU = reinterpret_cast<uint16_t*>(wsb + P.off_scaled);
 
-  // U = X A^T (fp32, optionally saved) and bf16(s * U) for the K extension
+  // LoRA dropout: the low-rank branch reads M * X (exact in bf16); c is applied to U
+  const uint16_t* Xl = X;
+  if (D.on) {
+    uint16_t* Xd = reinterpret_cast<uint16_t*>(wsb + P.total);
+    if (launch_dropout_mask(X, m * k, D.thr, D.seed, D.offset, Xd, D.mask, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    Xl = Xd;
+  }
+
+  // U = c (M * X) A^T (fp32, optionally saved) and bf16(s * U) for the K extension
   if (m <= 64) {
-    if (launch_lora_down_small(X, m, k, A, r, P.r_pad, s, U_save, sU, reinterpret_cast<float*>(wsb + P.off_part),
-                               st) != cudaSuccess)
+    if (launch_lora_down_small(Xl, m, k, A, r, P.r_pad, s, U_save, sU, reinterpret_cast<float*>(wsb + P.off_part),
+                               st, D.keep) != cudaSuccess)
       return QLORA_ERR_CUDA;
   } else {
-    const int rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st);
+    const int rc = run_lora_down(P, false, Xl, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st, D.keep);
     if (rc != QLORA_OK) return rc;
   }
 
@@ -503,6 +577,14 @@ int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, co
 int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t m, const uint16_t* A,
                      const uint16_t* B, int32_t r, float alpha, const float* U_saved, void* dX, int32_t dx_dtype,
                      float* dA, float* dB, int32_t flags, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  return qlora_linear_bwd_ex(w, X, dY, m, A, B, r, alpha, U_saved, dX, dx_dtype, dA, dB, flags, nullptr, ws,
+                             ws_bytes, stream);
+}
+
+int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* dY, int64_t m,
+                        const uint16_t* A, const uint16_t* B, int32_t r, float alpha, const float* U_saved,
+                        void* dX, int32_t dx_dtype, float* dA, float* dB, int32_t flags, const qlora_dropout* drop,
+                        void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (!linear_args_ok(w, X, m, A, B, r) || dY == nullptr || !aligned16(dY)) return QLORA_ERR_INVALID;
   if (dA == nullptr || dB == nullptr || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_INVALID;
   if (dX != nullptr && (!aligned16(dX) || (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_FP32)))
@@ -511,13 +593,23 @@ int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_
   if ((flags & ~(QLORA_BWD_ACCUMULATE_GRADS | QLORA_BWD_ACCUMULATE_DX)) != 0) return QLORA_ERR_INVALID;
   const int sst = linear_shape_status(w, r);
   if (sst != QLORA_OK) return sst;
+  Drop D;
+  if (resolve_drop(drop, &D) != QLORA_OK) return QLORA_ERR_INVALID;
   const int64_t n = w->n, k = w->k;
   const Plan P = make_plan(m, n, k, r);
-  if (ws == nullptr || !aligned16(ws) || ws_bytes < P.total) return QLORA_ERR_WORKSPACE;
+  const size_t need = P.total + (D.on ? drop_ws_bytes(m, k) : 0);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < need) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* wsb = static_cast<char*>(ws);
   const float s = alpha / static_cast<float>(r);
   uint16_t* sG = reinterpret_cast<uint16_t*>(wsb + P.off_scaled);
+  // LoRA dropout: M * X rebuilt from the forward's mask (dA and, without U_saved, U read it)
+  const uint16_t* Xl = X;
+  if (D.on) {
+    uint16_t* Xd = reinterpret_cast<uint16_t*>(wsb + P.total);
+    if (launch_mask_apply(X, m * k, D.mask, Xd, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    Xl = Xd;
+  }
   uint16_t* g_hi = reinterpret_cast<uint16_t*>(wsb + P.off_hi_b);
   uint16_t* g_lo = reinterpret_cast<uint16_t*>(wsb + P.off_lo_b);
   uint16_t* u_hi = reinterpret_cast<uint16_t*>(wsb + P.off_hi_a);
@@ -531,14 +623,14 @@ int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_
   if (U_saved != nullptr) {
     if (launch_split_hilo(U_saved, m, r, P.r_pad, u_hi, u_lo, st) != cudaSuccess) return QLORA_ERR_CUDA;
   } else {
-    rc = run_lora_down(P, false, X, m, k, A, r, s, wsb, nullptr, nullptr, u_hi, u_lo, st);
+    rc = run_lora_down(P, false, Xl, m, k, A, r, s, wsb, nullptr, nullptr, u_hi, u_lo, st, D.keep);
     if (rc != QLORA_OK) return rc;
   }
 
   if (dX != nullptr) {
     // dX^T = W^T . dY^T + A^T . (sG)^T, W dequantized into the MN-major operand layout
     GemmParams p = base_params(k, m, P.bn, cdiv(n, 64), P.bwd);
-    p.ext_tiles = P.r_pad / 64;
+    p.ext_tiles = D.on ? 0 : P.r_pad / 64;     // under dropout the low-rank term is added masked, below
     p.scales = scale_src(w);
     p.w_kblocks = k / 64;
     p.w_rows = static_cast<int32_t>(n);
@@ -567,11 +659,15 @@ int qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_
         launch_splitk_reduce(static_cast<const float*>(p.out), P.bwd.splits, p.part_stride, m, k, k, dX,
                              dx_dtype == QLORA_DTYPE_BF16, acc_dx, st) != cudaSuccess)
       return QLORA_ERR_CUDA;
+    if (D.on) {
+      rc = run_lora_up_masked(P, sG, m, k, A, r, D, dX, dx_dtype == QLORA_DTYPE_FP32, st);
+      if (rc != QLORA_OK) return rc;
+    }
   }
 
   rc = run_lora_grad(P, P.db, dY, m, n, u_hi, u_lo, r, s, dB, 0, acc_grads, wsb, st);
   if (rc != QLORA_OK) return rc;
-  rc = run_lora_grad(P, P.da, X, m, k, g_hi, g_lo, r, s, dA, 1, acc_grads, wsb, st);
+  rc = run_lora_grad(P, P.da, Xl, m, k, g_hi, g_lo, r, D.on ? s * D.keep : s, dA, 1, acc_grads, wsb, st);
   return rc;
 }
 

@@ -52,6 +52,8 @@ enum OutMode : int {
   kOutBF16 = 0,     // bf16 [rows, cols] with leading dimension ld_out
   kOutF32 = 1,      // fp32 [rows, cols]
   kOutPartial = 2,  // fp32 split-K partial: out + split * part_stride, [rows, ld_out]
+  kOutMaskAccBF16 = 3,  // bf16 out += keep_scale * D where the bit mask keeps the element (dropout dX)
+  kOutMaskAccF32 = 4,   // fp32 out, same
 };
 
 struct GemmParams {
@@ -71,6 +73,9 @@ struct GemmParams {
   int32_t out_mode;
   int32_t accumulate;          // kOutBF16/kOutF32: out += D
   Nf4Table tab;
+  // masked modes: bit (row * ld_out + col) of `mask` (bit e % 8 of byte e / 8) keeps the element
+  const uint8_t* mask;
+  float keep_scale;
 };
 
 struct GemmMaps {
@@ -138,10 +143,11 @@ int merge_tile_cols();
 cudaError_t launch_merge(const MergeParams& p, const MergeMaps& maps, int grid, bool out_f32, cudaStream_t st);
 
 // ------------------------------------------------------------- elementwise
+// U = pre * (sum of the split partials); writes fp32 U, bf16(scale * U), hi/lo bf16 of U (each nullable).
 cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
                                  int32_t r, int32_t r_pad, float scale, float* out_f32,
                                  uint16_t* out_scaled_bf16, uint16_t* out_hi, uint16_t* out_lo,
-                                 cudaStream_t st);
+                                 cudaStream_t st, float pre = 1.0f);
 cudaError_t launch_split_hilo(const float* src, int64_t rows, int32_t r, int32_t r_pad, uint16_t* hi,
                               uint16_t* lo, cudaStream_t st);
 cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
@@ -156,7 +162,11 @@ cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_str
 int lora_down_small_slices(int64_t k);
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
                                    int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
-                                   cudaStream_t st);
+                                   cudaStream_t st, float pre = 1.0f);
+// LoRA dropout (dropout.cu): keep mask from Philox4x32-10, masked copy of X, packed mask bits.
+cudaError_t launch_dropout_mask(const uint16_t* X, int64_t count, uint32_t thr, uint64_t seed, uint64_t offset,
+                                uint16_t* Xd, uint8_t* mask, cudaStream_t st);
+cudaError_t launch_mask_apply(const uint16_t* X, int64_t count, const uint8_t* mask, uint16_t* Xd, cudaStream_t st);
 cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
                                  cudaStream_t st);

@@ -210,6 +210,51 @@ int qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_
                      void *dX, int32_t dx_dtype, float *dA, float *dB, int32_t flags, void *ws,
                      size_t ws_bytes, qlora_stream_t stream);
 
+/*
+ * LoRA dropout on the input of the low-rank branch ("QLoRA Explained", Step 3:
+ * LoraConfig lora_dropout = 0.05; hyperparameter quick reference). The pages
+ * give only the rate; this library applies inverted dropout the way PEFT
+ * does: the branch sees M * X, with keep mask M, and its output is scaled by
+ * c = 1 / (1 - p). So U = c (M * X) A^T, dA = (alpha/r) c (dY B)^T (M * X),
+ * and dX gets (alpha/r) c ((dY B) A) * M.
+ *  - M comes from Philox4x32-10 (Salmon et al., SC 2011):
+ *      counter = (e / 8 as two 32-bit words, offset as two words),
+ *      key = seed as two words.
+ *    Element e of X (row-major) reads the 16-bit lane e % 8 of the four
+ *    output words (word (e % 8) / 2, low half first). It is kept iff that
+ *    value >= round(p * 65536). The effective rate is round(p * 65536) / 65536,
+ *    and c = 65536 / (65536 - round(p * 65536)).
+ *  - p in [0, 1); p = 0 disables dropout.
+ *  - mask: caller-owned device buffer of m * k / 8 bytes; element e is bit
+ *    e % 8 of byte e / 8. The forward writes it. The backward reads it and
+ *    does not draw again, so pass the same buffer (or the same bytes) to both.
+ *  - Vary seed or offset per step to get a fresh mask.
+ */
+typedef struct {
+  float p;
+  int32_t reserved;
+  uint64_t seed;
+  uint64_t offset;
+  uint8_t *mask;
+} qlora_dropout;
+
+/* Workspace for qlora_linear_fwd_ex / qlora_linear_bwd_ex. With dropout on,
+ * it holds a masked copy of X as well (m * k * 2 more bytes). */
+size_t qlora_linear_workspace_bytes_ex(int64_t m, int64_t n, int64_t k, int32_t r, const qlora_dropout *drop);
+
+/* qlora_linear_fwd with optional LoRA dropout (drop NULL or p == 0: identical to
+ * qlora_linear_fwd). U_save then holds U = c (M * X) A^T. Invalid p, or a NULL
+ * or misaligned mask with p > 0: QLORA_ERR_INVALID. */
+int qlora_linear_fwd_ex(const qlora_nf4_weight *w, const uint16_t *X, int64_t m, const uint16_t *A,
+                        const uint16_t *B, int32_t r, float alpha, void *Y, int32_t y_dtype, float *U_save,
+                        const qlora_dropout *drop, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* qlora_linear_bwd with optional LoRA dropout; drop->mask must hold the forward's mask. */
+int qlora_linear_bwd_ex(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t m,
+                        const uint16_t *A, const uint16_t *B, int32_t r, float alpha, const float *U_saved,
+                        void *dX, int32_t dx_dtype, float *dA, float *dB, int32_t flags,
+                        const qlora_dropout *drop, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
 /* SiLU-gated MLP glue (bf16 in/out, fp32 math): h = silu(g) * u. */
 int qlora_silu_gate_fwd(const uint16_t *g, const uint16_t *u, uint16_t *h, int64_t count, qlora_stream_t stream);
 

@@ -108,6 +108,17 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.qlora_lora_merge(ctypes.byref(ww), 1 << 24, 1 << 25, 12, 16.0, 1 << 26, 0, None) == 2
     wk = _weight(k=200)
     assert L.qlora_lora_merge(ctypes.byref(wk), 1 << 24, 1 << 25, 8, 16.0, 1 << 26, 1, None) == 2
+    # dropout: rate outside [0, 1), missing or misaligned mask; the workspace grows by m * k * 2
+    ww = _weight()
+    for p_, mask_ in ((1.5, 1 << 28), (-0.1, 1 << 28), (0.05, None), (0.05, (1 << 28) | 4)):
+        d = q.Dropout(p_, 1, 0, mask_)
+        rc = L.qlora_linear_fwd_ex(ctypes.byref(ww), 1 << 23, 128, 1 << 24, 1 << 25, 8, 16.0, 1 << 26, 0, None,
+                                   ctypes.byref(d), 1 << 27, 1 << 30, None)
+        assert rc == 1, (p_, mask_, rc)
+    base = q.qlora_linear_workspace_bytes(128, 256, 256, 8)
+    assert q.qlora_linear_workspace_bytes_ex(128, 256, 256, 8, None) == base
+    assert q.qlora_linear_workspace_bytes_ex(128, 256, 256, 8, q.Dropout(0.0, 1, 0, None)) == base
+    assert q.qlora_linear_workspace_bytes_ex(128, 256, 256, 8, q.Dropout(0.05, 1, 0, 1 << 28)) == base + 128 * 256 * 2
     # elementwise
     assert L.qlora_silu_gate_fwd(None, None, None, 16, None) == 1
     assert L.qlora_silu_gate_fwd(None, None, None, 0, None) == 0
