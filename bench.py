@@ -427,6 +427,30 @@ def components(dev, peaks) -> dict:
     algo = n * k * (0.5 + 1.0 / 64 + 4.0 / 16384) + 2.0 * M_SMALL * (k + n) + 2.0 * RANK_R * (k + n)
     out["fwd_m16_q_proj"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
                              "algo_bytes": algo}
+    # LoRA dropout (p = 0.05): q_proj forward + backward at 8192 tokens with and without it
+    M = M_TOKENS
+    X = synth.activations(M, k).to(dev)
+    dY = synth.grad_output(M, n).to(dev)
+    Yb = torch.empty(M, n, dtype=torch.bfloat16, device=dev)
+    dXb = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
+    Ub = torch.empty(M, RANK_R, dtype=torch.float32, device=dev)
+    dAb = torch.empty(RANK_R, k, dtype=torch.float32, device=dev)
+    dBb = torch.empty(n, RANK_R, dtype=torch.float32, device=dev)
+    mask = torch.empty(M * k // 8, dtype=torch.uint8, device=dev)
+    drop = q.Dropout(0.05, 1234, 0, mask)
+    wsd = torch.empty(q.qlora_linear_workspace_bytes_ex(M, n, k, RANK_R, drop), dtype=torch.uint8, device=dev)
+    times = {}
+    for tag, d in (("plain", None), ("dropout", drop)):
+        def fb(d=d):
+            q.qlora_linear_fwd_ex(qw, X, a, b, RANK_R, ALPHA, Yb, q.QLORA_DTYPE_BF16, Ub, d, wsd)
+            q.qlora_linear_bwd_ex(qw, X, dY, a, b, RANK_R, ALPHA, Ub, dXb, q.QLORA_DTYPE_BF16, dAb, dBb, 0, d, wsd)
+        for _ in range(2):
+            fb()
+        times[tag] = graph_time(fb, 3, flush)
+    out["dropout_fwd_bwd_q_proj"] = {"us": times["dropout"] * 1e3, "us_without": times["plain"] * 1e3,
+                                     "overhead": times["dropout"] / times["plain"] - 1.0, "p": 0.05,
+                                     "tokens": M}
+    del X, dY, Yb, dXb, wsd
     # adapter merge onto the dequantized weight (65B q_proj, bf16 output)
     wm = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
     fn = lambda: q.qlora_lora_merge(qw, a, b, RANK_R, ALPHA, wm, q.QLORA_DTYPE_BF16)
@@ -472,6 +496,27 @@ def run_case(args) -> None:
                 q.qlora_linear_bwd(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, ws)
             else:
                 q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+    elif name == "dropout_q_65b":
+        n, k = LAYERS[0][1], LAYERS[0][2]
+        m = M_TOKENS
+        W = synth.weight(n, k).to(dev)
+        qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+        q.qlora_nf4_quantize(W, qw)
+        del W
+        a, b = (t.to(dev) for t in synth.lora_pair(RANK_R, k, n))
+        x = synth.activations(m, k).to(dev)
+        dy = synth.grad_output(m, n).to(dev)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+        dx = torch.empty(m, k, dtype=torch.bfloat16, device=dev)
+        u = torch.empty(m, RANK_R, dtype=torch.float32, device=dev)
+        da = torch.empty(RANK_R, k, dtype=torch.float32, device=dev)
+        db = torch.empty(n, RANK_R, dtype=torch.float32, device=dev)
+        mask = torch.empty(m * k // 8, dtype=torch.uint8, device=dev)
+        drop = q.Dropout(0.05, 1234, 0, mask)
+        ws = torch.empty(q.qlora_linear_workspace_bytes_ex(m, n, k, RANK_R, drop), dtype=torch.uint8, device=dev)
+        for _ in range(1 + args.case_iters):
+            q.qlora_linear_fwd_ex(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, drop, ws)
+            q.qlora_linear_bwd_ex(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, drop, ws)
     elif name == "merge_q_65b":
         n, k = LAYERS[0][1], LAYERS[0][2]
         W = synth.weight(n, k).to(dev)

@@ -37,7 +37,8 @@ struct GemmCfg {
   static constexpr int kThreads = 6 * 32;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = Stages * (kABytes + kBBytes) + 1024 + kBarBytes;
+  static constexpr int kEpiStage = 4 * 32 * 32 * 4;   // one 32 x 32 fp32 chunk per epilogue warp (masked modes)
+  static constexpr int kSmemBytes = Stages * (kABytes + kBBytes) + kEpiStage + 1024 + kBarBytes;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM alloc size");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -82,47 +83,6 @@ __device__ __forceinline__ void store_row32(const GemmParams& p, int split, int 
     return;
   }
   const bool full = (col0 + 32 <= p.cols);
-  if (p.out_mode == kOutMaskAccBF16 || p.out_mode == kOutMaskAccF32) {
-    // dropout dX: out += keep_scale * D where the mask keeps the element (the 32 columns start on a
-    // multiple of 32 of a row whose length is a multiple of 64, so their bits are one aligned word)
-    const int64_t e0 = static_cast<int64_t>(row) * p.ld_out + col0;
-    const uint32_t bits = __ldg(reinterpret_cast<const uint32_t*>(p.mask + e0 / 8));
-    if (p.out_mode == kOutMaskAccF32) {
-      float* o = static_cast<float*>(p.out) + e0;
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        float4 y = *reinterpret_cast<const float4*>(o + j);
-        y.x += ((bits >> j) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j])) : 0.f;
-        y.y += ((bits >> (j + 1)) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j + 1])) : 0.f;
-        y.z += ((bits >> (j + 2)) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j + 2])) : 0.f;
-        y.w += ((bits >> (j + 3)) & 1u) ? __fmul_rn(p.keep_scale, __uint_as_float(v[j + 3])) : 0.f;
-        *reinterpret_cast<float4*>(o + j) = y;
-      }
-    } else {
-      uint16_t* o = static_cast<uint16_t*>(p.out) + e0;
-#pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        const uint4 y = *reinterpret_cast<const uint4*>(o + j);
-        const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
-        float x[8];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          x[2 * t] = __uint_as_float(yy[t] << 16);
-          x[2 * t + 1] = __uint_as_float(yy[t] & 0xFFFF0000u);
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          if ((bits >> (j + t)) & 1u) x[t] += __fmul_rn(p.keep_scale, __uint_as_float(v[j + t]));
-        uint4 w;
-        w.x = pack_bf16x2(x[0], x[1]);
-        w.y = pack_bf16x2(x[2], x[3]);
-        w.z = pack_bf16x2(x[4], x[5]);
-        w.w = pack_bf16x2(x[6], x[7]);
-        *reinterpret_cast<uint4*>(o + j) = w;
-      }
-    }
-    return;
-  }
   if (p.out_mode == kOutF32) {
     float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.ld_out + col0;
     if (full) {
@@ -178,6 +138,87 @@ __device__ __forceinline__ void store_row32(const GemmParams& p, int split, int 
   }
 }
 
+// Masked accumulate (dropout dX) of one warp's 32 rows x NCH*32 columns of a unit:
+// out += keep_scale * D where the mask bit of the element is set. Every output vector
+// and mask byte of the unit is requested first (one memory round trip per unit); then
+// each 32-column chunk of the accumulator goes through a 128B-swizzled fp32 staging tile
+// so that four lanes share one output row and every access covers 8 rows x 64 bytes.
+template <int NCH>
+__device__ __forceinline__ void masked_acc_unit(const GemmParams& p, uint32_t stage, int lane, int row0, int col0,
+                                                uint32_t t_row) {
+  const int sub = lane >> 2;            // row within a pass of 8 rows
+  const int cc = (lane & 3) * 8;        // first of this lane's eight columns within a chunk
+  const bool f32 = (p.out_mode == kOutMaskAccF32);
+  uint4 y[NCH][4], y2[NCH][4];
+  uint32_t bits[NCH][4];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int row = row0 + pass * 8 + sub;
+      y[c][pass] = y2[c][pass] = make_uint4(0u, 0u, 0u, 0u);
+      bits[c][pass] = 0u;
+      // a group of eight columns lies wholly inside or wholly outside the row (cols % 64 == 0)
+      if (row < p.rows && col0 + c * 32 + cc < p.cols) {
+        const int64_t e0 = static_cast<int64_t>(row) * p.ld_out + col0 + c * 32 + cc;   // a multiple of 8
+        bits[c][pass] = __ldg(p.mask + e0 / 8);
+        if (f32) {
+          const uint4* o = reinterpret_cast<const uint4*>(static_cast<const float*>(p.out) + e0);
+          y[c][pass] = o[0];
+          y2[c][pass] = o[1];
+        } else {
+          y[c][pass] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.out) + e0);
+        }
+      }
+    }
+  const uint32_t mine = stage + lane * 128;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(t_row + c * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      st_shared_v4(mine + ((j ^ (lane & 7)) << 4), make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int rr = pass * 8 + sub;
+      const int row = row0 + rr;
+      if (row >= p.rows || col0 + c * 32 + cc >= p.cols) continue;
+      const uint32_t src = stage + rr * 128;
+      const uint4 a0 = ld_shared_v4(src + (((cc >> 2) ^ (rr & 7)) << 4));
+      const uint4 a1 = ld_shared_v4(src + ((((cc >> 2) + 1) ^ (rr & 7)) << 4));
+      const float d[8] = {__uint_as_float(a0.x), __uint_as_float(a0.y), __uint_as_float(a0.z), __uint_as_float(a0.w),
+                          __uint_as_float(a1.x), __uint_as_float(a1.y), __uint_as_float(a1.z), __uint_as_float(a1.w)};
+      float add[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) add[t] = ((bits[c][pass] >> t) & 1u) ? __fmul_rn(p.keep_scale, d[t]) : 0.f;
+      const int64_t e0 = static_cast<int64_t>(row) * p.ld_out + col0 + c * 32 + cc;
+      if (f32) {
+        uint4* o = reinterpret_cast<uint4*>(static_cast<float*>(p.out) + e0);
+        o[0] = make_uint4(__float_as_uint(__uint_as_float(y[c][pass].x) + add[0]),
+                          __float_as_uint(__uint_as_float(y[c][pass].y) + add[1]),
+                          __float_as_uint(__uint_as_float(y[c][pass].z) + add[2]),
+                          __float_as_uint(__uint_as_float(y[c][pass].w) + add[3]));
+        o[1] = make_uint4(__float_as_uint(__uint_as_float(y2[c][pass].x) + add[4]),
+                          __float_as_uint(__uint_as_float(y2[c][pass].y) + add[5]),
+                          __float_as_uint(__uint_as_float(y2[c][pass].z) + add[6]),
+                          __float_as_uint(__uint_as_float(y2[c][pass].w) + add[7]));
+      } else {
+        const uint32_t yy[4] = {y[c][pass].x, y[c][pass].y, y[c][pass].z, y[c][pass].w};
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[t] = pack_bf16x2(__uint_as_float(yy[t] << 16) + add[2 * t],
+                             __uint_as_float(yy[t] & 0xFFFF0000u) + add[2 * t + 1]);
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + e0) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    __syncwarp();                       // the staging tile is rewritten by the next chunk
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1)
     qlora_gemm_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmMaps maps) {
@@ -186,7 +227,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::Stages * C::kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::Stages * C::kBBytes);
+  uint8_t* sEpi = sB + C::Stages * C::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + C::kEpiStage);
   uint64_t* tma_full = bars;
   uint64_t* empty = bars + C::Stages;
   uint64_t* acc_full = bars + 2 * C::Stages;
@@ -340,12 +382,16 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       tc_fence_after();
       const int row = mb * 128 + q * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+      if (p.out_mode == kOutMaskAccBF16 || p.out_mode == kOutMaskAccF32) {
+        masked_acc_unit<C::BN / 32>(p, smem_u32(sEpi + q * 4096), lane, mb * 128 + q * 32, nb * C::BN, t_row);
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
-        tmem_ld_wait();
-        store_row32(p, split, row, nb * C::BN + c * 32, v);
+        for (int c = 0; c < C::BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_row + c * 32, v);
+          tmem_ld_wait();
+          store_row32(p, split, row, nb * C::BN + c * 32, v);
+        }
       }
       tc_fence_before();
       __syncwarp();
