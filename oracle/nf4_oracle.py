@@ -71,6 +71,14 @@ design notes of the repository):
    e % 8 of the four output words (word (e % 8) // 2, low half first) and is
    kept iff that value >= round(p * 65536). The effective drop rate is
    round(p * 65536) / 65536 and c = 65536 / (65536 - round(p * 65536)).
+11. Paged AdamW, 32-bit ([GAMUT] "Paged Optimizers" and the hyperparameter
+   reference, optim="paged_adamw_32bit"; [CSD] "Paged optimizers (the
+   storage unit)"): AdamW with decoupled weight decay (Loshchilov and Hutter)
+   on fp32 master weights of the adapters with fp32 moment estimates:
+   g = grad * grad_scale; m = b1 m + (1 - b1) g; v = b2 v + (1 - b2) g^2;
+   p = p (1 - lr wd) - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps).
+   "Paged" is where the states live (unified memory that may spill to host
+   RAM), not a change to the arithmetic.
 """
 from __future__ import annotations
 
@@ -459,6 +467,21 @@ def linear_backward_dropout(Wd, X, dY, A, B, alpha: float, mask, p: float, dx_ro
     else:
         dX = dY @ Wd + s * c * ((G @ A) * Mf)
     return dX, dA, dB
+
+
+# ----------------------------------------------------------------------------
+# AdamW on the adapter masters (reading 11), fp64
+# ----------------------------------------------------------------------------
+def adamw_step(param, grad, m, v, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+               eps: float = 1e-8, weight_decay: float = 0.0, grad_scale: float = 1.0):
+    """One AdamW step (decoupled weight decay) in fp64; returns (param, m, v)."""
+    p, g, m, v = _f64(param), _f64(grad) * grad_scale, _f64(m), _f64(v)
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    bc1 = 1.0 - beta1 ** step
+    bc2 = 1.0 - beta2 ** step
+    p = p * (1.0 - lr * weight_decay) - (lr / bc1) * m / (np.sqrt(v) / math.sqrt(bc2) + eps)
+    return p, m, v
 
 
 def silu_gate_forward(g, u):

@@ -498,3 +498,41 @@ def test_mask_bit_packing_order():
     mask = np.zeros((2, 16), dtype=bool)
     mask[0, 0] = mask[0, 9] = mask[1, 15] = True
     assert o.pack_mask_bits(mask).tolist() == [0x01, 0x02, 0x00, 0x80]
+
+
+# ------------------------------------------------------------------- AdamW
+def test_adamw_first_step_is_a_sign_step():
+    # with zero moments the bias-corrected first step is lr * g / (|g| + eps): a sign step for |g| >> eps
+    rng = np.random.default_rng(21)
+    p0, g = rng.normal(0, 1, 1000), rng.normal(0, 1e-2, 1000)
+    p1, m1, v1 = o.adamw_step(p0, g, np.zeros(1000), np.zeros(1000), step=1, lr=2e-4, eps=1e-8)
+    np.testing.assert_allclose(p1, p0 - 2e-4 * g / (np.abs(g) + 1e-8), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(m1, 0.1 * g, rtol=1e-15)
+    np.testing.assert_allclose(v1, 0.001 * g * g, rtol=1e-12)
+
+
+def test_adamw_constant_gradient_closed_form():
+    # a constant gradient keeps the bias-corrected moments at g and g^2 for every t, so each step
+    # moves by lr * g / (|g| + eps); with weight decay the parameter follows a geometric recursion
+    g, lr, wd, eps, T = np.array([3e-3, -2e-2, 5e-1]), 1e-3, 0.01, 1e-8, 25
+    p = np.array([0.5, -1.0, 2.0])
+    m = np.zeros(3)
+    v = np.zeros(3)
+    for t in range(1, T + 1):
+        p, m, v = o.adamw_step(p, g, m, v, step=t, lr=lr, weight_decay=wd, eps=eps)
+    u = lr * g / (np.abs(g) + eps)
+    a = 1 - lr * wd
+    want = np.array([0.5, -1.0, 2.0]) * a ** T - u * (1 - a ** T) / (1 - a)
+    np.testing.assert_allclose(p, want, rtol=1e-10)
+
+
+def test_adamw_zero_gradient_only_decays():
+    p0 = np.array([1.0, -2.0, 0.25])
+    p1, m1, v1 = o.adamw_step(p0, np.zeros(3), np.zeros(3), np.zeros(3), step=3, lr=0.1, weight_decay=0.5)
+    np.testing.assert_allclose(p1, p0 * (1 - 0.05), rtol=1e-15)
+    assert np.all(m1 == 0) and np.all(v1 == 0)
+    # grad_scale multiplies the gradient before anything else
+    a = o.adamw_step(p0, np.full(3, 2.0), np.zeros(3), np.zeros(3), step=1, lr=0.1, grad_scale=0.5)
+    b = o.adamw_step(p0, np.full(3, 1.0), np.zeros(3), np.zeros(3), step=1, lr=0.1)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
