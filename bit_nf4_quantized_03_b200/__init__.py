@@ -36,6 +36,7 @@ EXPORTED = (
     "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end",
     "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
+    "qlora_adamw_step", "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch",
 )
 
 
@@ -69,6 +70,19 @@ class Dropout(ctypes.Structure):
     def __init__(self, p: float, seed: int, offset: int, mask):
         super().__init__(float(p), 0, int(seed), int(offset), _ptr(mask))
         self._mask = mask
+
+
+class AdamWConfig(ctypes.Structure):
+    """Mirror of qlora_adamw_config."""
+    _fields_ = [
+        ("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+        ("weight_decay", ctypes.c_float), ("grad_scale", ctypes.c_float), ("step", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+    def __init__(self, lr: float, step: int, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                 weight_decay: float = 0.0, grad_scale: float = 1.0):
+        super().__init__(lr, beta1, beta2, eps, weight_decay, grad_scale, int(step), 0)
 
 
 _lib = None
@@ -106,6 +120,10 @@ def lib() -> ctypes.CDLL:
         "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
         "qlora_linear_workspace_bytes_ex": (sz, [i64, i64, i64, i32, pd]),
+        "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWConfig), vp]),
+        "qlora_paged_alloc": (ctypes.c_int, [sz, ctypes.POINTER(ctypes.c_void_p)]),
+        "qlora_paged_free": (ctypes.c_int, [vp]),
+        "qlora_paged_prefetch": (ctypes.c_int, [vp, sz, i32, vp]),
         "qlora_linear_fwd_ex": (ctypes.c_int, [pw, vp, i64, vp, vp, i32, f32, vp, i32, vp, pd, vp, sz, vp]),
         "qlora_linear_bwd_ex": (ctypes.c_int, [pw, vp, vp, i64, vp, vp, i32, f32, vp, vp, i32, vp, vp, i32,
                                                pd, vp, sz, vp]),
@@ -265,6 +283,28 @@ def qlora_linear_bwd_ex(w: QuantizedWeight, X, dY, A, B, r: int, alpha: float, U
                                    _ptr(U_saved), _ptr(dX), dx_dtype, _ptr(dA), _ptr(dB), flags, _dref(drop),
                                    _ptr(ws), ws_bytes, _stream(stream))
     _check(rc, "qlora_linear_bwd_ex")
+
+
+def qlora_adamw_step(param, grad, m, v, param_bf16, count: int, cfg: AdamWConfig, stream=None):
+    """One AdamW step on fp32 masters (tensors or device-accessible addresses)."""
+    _check(lib().qlora_adamw_step(_ptr(param), _ptr(grad), _ptr(m), _ptr(v), _ptr(param_bf16), int(count),
+                                  ctypes.byref(cfg), _stream(stream)), "qlora_adamw_step")
+
+
+def qlora_paged_alloc(nbytes: int) -> int:
+    """Managed (pageable unified) memory for optimizer states; returns its address."""
+    out = ctypes.c_void_p(0)
+    _check(lib().qlora_paged_alloc(int(nbytes), ctypes.byref(out)), "qlora_paged_alloc")
+    return int(out.value)
+
+
+def qlora_paged_free(addr: int):
+    _check(lib().qlora_paged_free(addr), "qlora_paged_free")
+
+
+def qlora_paged_prefetch(addr: int, nbytes: int, to_host: bool = False, stream=None):
+    _check(lib().qlora_paged_prefetch(addr, int(nbytes), 1 if to_host else 0, _stream(stream)),
+           "qlora_paged_prefetch")
 
 
 def qlora_silu_gate_fwd(g, u, h, stream=None):

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libqlora.so")
-SOURCES = ["nf4_quant.cu", "nf4_gemm.cu", "nf4_wgemm.cu", "elementwise.cu", "qlora_abi.cu", "nf4_merge.cu", "dropout.cu", "qlora_noalloc.cu"]
+SOURCES = ["nf4_quant.cu", "nf4_gemm.cu", "nf4_wgemm.cu", "elementwise.cu", "qlora_abi.cu", "nf4_merge.cu", "dropout.cu", "optim.cu", "qlora_noalloc.cu"]
 HEADERS = ["qlora_device.cuh", "qlora_kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-Xcompiler", "-fPIC",

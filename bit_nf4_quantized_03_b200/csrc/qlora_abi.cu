@@ -672,6 +672,54 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
   return rc;
 }
 
+int qlora_adamw_step(float* param, const float* grad, float* m, float* v, uint16_t* param_bf16, int64_t count,
+                     const qlora_adamw_config* cfg, qlora_stream_t stream) {
+  if (cfg == nullptr || count < 0) return QLORA_ERR_INVALID;
+  if (count == 0) return QLORA_OK;
+  if (param == nullptr || grad == nullptr || m == nullptr || v == nullptr) return QLORA_ERR_INVALID;
+  if (!aligned16(param) || !aligned16(grad) || !aligned16(m) || !aligned16(v)) return QLORA_ERR_INVALID;
+  if (param_bf16 != nullptr && (reinterpret_cast<uintptr_t>(param_bf16) & 7u) != 0) return QLORA_ERR_INVALID;
+  if (cfg->step < 1 || !(cfg->beta1 > 0.f && cfg->beta1 < 1.f) || !(cfg->beta2 > 0.f && cfg->beta2 < 1.f) ||
+      !(cfg->eps > 0.f) || !std::isfinite(cfg->lr) || !std::isfinite(cfg->weight_decay) ||
+      !std::isfinite(cfg->grad_scale))
+    return QLORA_ERR_INVALID;
+  return cuda_status(launch_adamw(param, grad, m, v, param_bf16, count, cfg->lr, cfg->beta1, cfg->beta2, cfg->eps,
+                                  cfg->weight_decay, cfg->grad_scale, cfg->step, num_sms(),
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_paged_alloc(size_t bytes, void** out) {
+  if (out == nullptr || bytes == 0) return QLORA_ERR_INVALID;
+  *out = nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  void* ptr = nullptr;
+  if (cudaMallocManaged(&ptr, bytes, cudaMemAttachGlobal) != cudaSuccess) return QLORA_ERR_CUDA;
+  // home on the current device; the driver may still migrate pages to host RAM under pressure
+  cudaMemLocation loc;
+  loc.type = cudaMemLocationTypeDevice;
+  loc.id = dev;
+  (void)cudaMemAdvise(ptr, bytes, cudaMemAdviseSetPreferredLocation, loc);
+  (void)cudaGetLastError();      // the advice is a hint: a device without it still works
+  *out = ptr;
+  return QLORA_OK;
+}
+
+int qlora_paged_free(void* ptr) {
+  if (ptr == nullptr) return QLORA_OK;
+  return cuda_status(cudaFree(ptr));
+}
+
+int qlora_paged_prefetch(const void* ptr, size_t bytes, int32_t to_host, qlora_stream_t stream) {
+  if (ptr == nullptr || bytes == 0) return QLORA_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  cudaMemLocation loc;
+  loc.type = to_host ? cudaMemLocationTypeHost : cudaMemLocationTypeDevice;
+  loc.id = to_host ? 0 : dev;
+  return cuda_status(cudaMemPrefetchAsync(ptr, bytes, loc, 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qlora_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count, qlora_stream_t stream) {
   if (count < 0) return QLORA_ERR_INVALID;
   if (count == 0) return QLORA_OK;

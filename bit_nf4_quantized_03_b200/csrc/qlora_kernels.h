@@ -167,6 +167,10 @@ cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, cons
 cudaError_t launch_dropout_mask(const uint16_t* X, int64_t count, uint32_t thr, uint64_t seed, uint64_t offset,
                                 uint16_t* Xd, uint8_t* mask, cudaStream_t st);
 cudaError_t launch_mask_apply(const uint16_t* X, int64_t count, const uint8_t* mask, uint16_t* Xd, cudaStream_t st);
+// AdamW step on fp32 masters (optim.cu); p_bf16 (nullable) receives bf16(p).
+cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, uint16_t* p_bf16, int64_t count, float lr,
+                         float beta1, float beta2, float eps, float weight_decay, float grad_scale, int32_t step,
+                         int num_sms, cudaStream_t st);
 cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
                                  cudaStream_t st);

@@ -255,6 +255,43 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight *w, const uint16_t *X, const uint
                         void *dX, int32_t dx_dtype, float *dA, float *dB, int32_t flags,
                         const qlora_dropout *drop, void *ws, size_t ws_bytes, qlora_stream_t stream);
 
+/*
+ * Paged AdamW, 32-bit, for the adapters ("QLoRA Explained": Paged Optimizers
+ * and optim = "paged_adamw_32bit"; "QLoRA: Quantized Low-Rank Adaptation":
+ * "Paged optimizers (the storage unit)"). AdamW with decoupled weight decay
+ * on fp32 masters and fp32 moments, one fused pass per parameter array:
+ *   g = grad * grad_scale;  m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2
+ *   p = p (1 - lr wd) - (lr / (1 - b1^step)) m / (sqrt(v) / sqrt(1 - b2^step) + eps)
+ * and, when param_bf16 is not NULL, param_bf16 = bf16(p) (the copy the GEMMs
+ * read). All arrays hold `count` elements, are 16-byte aligned and device
+ * accessible: device memory or qlora_paged_alloc memory. step >= 1;
+ * 0 < b1, b2 < 1; eps > 0; else QLORA_ERR_INVALID with nothing enqueued.
+ */
+typedef struct {
+  float lr;
+  float beta1;
+  float beta2;
+  float eps;
+  float weight_decay;
+  float grad_scale;
+  int32_t step;
+  int32_t reserved;
+} qlora_adamw_config;
+
+int qlora_adamw_step(float *param, const float *grad, float *m, float *v, uint16_t *param_bf16, int64_t count,
+                     const qlora_adamw_config *cfg, qlora_stream_t stream);
+
+/* Paged memory for optimizer states: unified (managed) memory with the
+ * current device as its preferred home. The driver may move it to host RAM
+ * when device memory runs short; qlora_paged_prefetch moves it explicitly
+ * (to_host = 0: to the current device, before the step; 1: to host RAM,
+ * freeing device memory during a spike). The allocation is the caller's and
+ * must be released with qlora_paged_free. These calls, unlike the compute
+ * entry points, allocate. */
+int qlora_paged_alloc(size_t bytes, void **out);
+int qlora_paged_free(void *ptr);
+int qlora_paged_prefetch(const void *ptr, size_t bytes, int32_t to_host, qlora_stream_t stream);
+
 /* SiLU-gated MLP glue (bf16 in/out, fp32 math): h = silu(g) * u. */
 int qlora_silu_gate_fwd(const uint16_t *g, const uint16_t *u, uint16_t *h, int64_t count, qlora_stream_t stream);
 

@@ -119,6 +119,19 @@ def test_invalid_arguments_rejected_on_host(L):
     assert q.qlora_linear_workspace_bytes_ex(128, 256, 256, 8, None) == base
     assert q.qlora_linear_workspace_bytes_ex(128, 256, 256, 8, q.Dropout(0.0, 1, 0, None)) == base
     assert q.qlora_linear_workspace_bytes_ex(128, 256, 256, 8, q.Dropout(0.05, 1, 0, 1 << 28)) == base + 128 * 256 * 2
+    # AdamW: bad hyperparameters or step, misaligned arrays; count 0 is a no-op
+    good = q.AdamWConfig(lr=2e-4, step=1)
+    args = (1 << 20, 1 << 21, 1 << 22, 1 << 23, None, 100)
+    assert L.qlora_adamw_step(*args[:5], 0, ctypes.byref(good), None) == 0
+    for bad in (q.AdamWConfig(lr=2e-4, step=0), q.AdamWConfig(lr=2e-4, step=1, beta1=1.0),
+                q.AdamWConfig(lr=2e-4, step=1, beta2=0.0), q.AdamWConfig(lr=2e-4, step=1, eps=0.0),
+                q.AdamWConfig(lr=float("nan"), step=1)):
+        assert L.qlora_adamw_step(*args, ctypes.byref(bad), None) == 1
+    assert L.qlora_adamw_step((1 << 20) | 4, *args[1:], ctypes.byref(good), None) == 1
+    assert L.qlora_adamw_step(*args[:4], (1 << 24) | 2, 100, ctypes.byref(good), None) == 1
+    assert L.qlora_adamw_step(*args, None, None) == 1
+    assert L.qlora_paged_free(None) == 0
+    assert L.qlora_paged_prefetch(None, 16, 0, None) == 1
     # elementwise
     assert L.qlora_silu_gate_fwd(None, None, None, 16, None) == 1
     assert L.qlora_silu_gate_fwd(None, None, None, 0, None) == 0
