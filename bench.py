@@ -451,6 +451,49 @@ def components(dev, peaks) -> dict:
                                      "overhead": times["dropout"] / times["plain"] - 1.0, "p": 0.05,
                                      "tokens": M}
     del X, dY, Yb, dXb, wsd
+    # paged AdamW over one decoder layer's adapters (r = 64: q/k/v/o 64 x (8192 + 8192), gate/up/down
+    # 64 x (8192 + 22016)); 30 bytes per parameter: p, g, m, v read; p, m, v and the bf16 copy written
+    count = sum(RANK_R * (nn + kk) for _, nn, kk in LAYERS)
+    algo = 30.0 * count
+    grad = torch.randn(count, device=dev) * 1e-2
+    pbf = torch.empty(count, dtype=torch.bfloat16, device=dev)
+    dev_states = [torch.zeros(count, device=dev) for _ in range(3)]
+    cfg = q.AdamWConfig(2e-4, 10, weight_decay=0.01)
+    fn = lambda: q.qlora_adamw_step(dev_states[0], grad, dev_states[1], dev_states[2], pbf, count, cfg)
+    for _ in range(3):
+        fn()
+    ms = graph_time(fn, 20, flush)
+    out["adamw_layer_adapters"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
+                                   "algo_bytes": algo, "params": count}
+    nbytes = count * 4
+    addrs = [q.qlora_paged_alloc(nbytes) for _ in range(3)]
+    try:
+        for addr in addrs:
+            q.qlora_paged_prefetch(addr, nbytes)
+        fnp = lambda: q.qlora_adamw_step(addrs[0], grad, addrs[1], addrs[2], pbf, count, cfg)
+        for _ in range(3):
+            fnp()
+        msp = graph_time(fnp, 20, flush)
+        # page the three state arrays out to host RAM and back in (the paging cost of one step)
+        torch.cuda.synchronize()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        for addr in addrs:
+            q.qlora_paged_prefetch(addr, nbytes, to_host=True)
+        e1.record()
+        for addr in addrs:
+            q.qlora_paged_prefetch(addr, nbytes)
+        e2.record()
+        torch.cuda.synchronize()
+        out["adamw_layer_adapters_paged"] = {
+            "us": msp * 1e3, "gbs": algo / msp / 1e6, "frac": algo / msp / 1e6 / peaks["hbm_gbs"],
+            "algo_bytes": algo, "params": count, "page_out_us": e0.elapsed_time(e1) * 1e3,
+            "page_in_us": e1.elapsed_time(e2) * 1e3, "paged_bytes": 3 * nbytes}
+    finally:
+        torch.cuda.synchronize()
+        for addr in addrs:
+            q.qlora_paged_free(addr)
+    del grad, pbf, dev_states
     # adapter merge onto the dequantized weight (65B q_proj, bf16 output)
     wm = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
     fn = lambda: q.qlora_lora_merge(qw, a, b, RANK_R, ALPHA, wm, q.QLORA_DTYPE_BF16)

@@ -68,7 +68,7 @@ class Dropout(ctypes.Structure):
     ]
 
     def __init__(self, p: float, seed: int, offset: int, mask):
-        super().__init__(float(p), 0, int(seed), int(offset), _ptr(mask))
+        super().__init__(float(p), 0, int(seed), int(offset), _ptr(mask, allow_addr=True))
         self._mask = mask
 
 
@@ -140,10 +140,15 @@ def status_string(status: int) -> str:
     return lib().qlora_status_string(int(status)).decode()
 
 
-def _ptr(t) -> int | None:
+def _ptr(t, allow_addr: bool = False) -> int | None:
+    """Device address of a CUDA tensor. Raw integer addresses are accepted only where
+    an entry point documents them (paged memory), so a stray integer cannot stand in
+    for a tensor argument."""
     if t is None:
         return None
     if isinstance(t, int):
+        if not allow_addr:
+            raise TypeError("expected a CUDA tensor, got an integer address")
         return t
     if not t.is_cuda:
         raise ValueError("libqlora takes CUDA tensors only (no CPU fallback)")
@@ -287,8 +292,9 @@ def qlora_linear_bwd_ex(w: QuantizedWeight, X, dY, A, B, r: int, alpha: float, U
 
 def qlora_adamw_step(param, grad, m, v, param_bf16, count: int, cfg: AdamWConfig, stream=None):
     """One AdamW step on fp32 masters (tensors or device-accessible addresses)."""
-    _check(lib().qlora_adamw_step(_ptr(param), _ptr(grad), _ptr(m), _ptr(v), _ptr(param_bf16), int(count),
-                                  ctypes.byref(cfg), _stream(stream)), "qlora_adamw_step")
+    _check(lib().qlora_adamw_step(_ptr(param, True), _ptr(grad, True), _ptr(m, True), _ptr(v, True),
+                                  _ptr(param_bf16, True), int(count), ctypes.byref(cfg), _stream(stream)),
+           "qlora_adamw_step")
 
 
 def qlora_paged_alloc(nbytes: int) -> int:

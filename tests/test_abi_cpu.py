@@ -143,3 +143,7 @@ def test_binding_refuses_cpu_tensors(L):
     w = torch.zeros(64, 64)
     with pytest.raises(ValueError):
         q._ptr(w)
+    # an integer stands in for a tensor only where an entry point documents raw addresses
+    with pytest.raises(TypeError):
+        q._ptr(1 << 20)
+    assert q._ptr(1 << 20, allow_addr=True) == 1 << 20
