@@ -615,6 +615,13 @@ def run_case(args) -> None:
         for _ in range(1 + args.case_iters):
             q.qlora_linear_fwd_ex(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, drop, ws)
             q.qlora_linear_bwd_ex(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, drop, ws)
+    elif name == "adamw_layer":
+        count = sum(RANK_R * (nn + kk) for _, nn, kk in LAYERS)
+        grad = torch.randn(count, device=dev) * 1e-2
+        pbf = torch.empty(count, dtype=torch.bfloat16, device=dev)
+        st = [torch.zeros(count, device=dev) for _ in range(3)]
+        for t in range(1 + args.case_iters):
+            q.qlora_adamw_step(st[0], grad, st[1], st[2], pbf, count, q.AdamWConfig(2e-4, t + 1, weight_decay=0.01))
     elif name == "merge_q_65b":
         n, k = LAYERS[0][1], LAYERS[0][2]
         W = synth.weight(n, k).to(dev)
