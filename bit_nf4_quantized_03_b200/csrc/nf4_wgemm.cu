@@ -22,6 +22,7 @@
 //               every K step of the 128-row tile
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "qlora_kernels.h"
@@ -56,6 +57,8 @@ struct WCfg {
 };
 
 constexpr int kRasterGroup = 4;   // token tiles per raster group (L2 reuse of both operands)
+constexpr int64_t kPair512From = 1024;   // above this many tokens a CTA pair takes 512 per unit
+
 
 __device__ __forceinline__ void wdecode(const GemmParams& p, int u, int& mb, int& nb, int& split, int& kt0,
                                         int& nmain, int& next) {
@@ -236,7 +239,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int i = 0; i < nmain + next; ++i) {
           if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
           if (!mbar_wait(&deq_full[stage], ph)) { ok = false; break; }
-          tc_fence_after();
+          // operands reach the MMA through the barriers alone (TMA completion; the
+          // dequantizers' fence.proxy.async before their arrival): no tcgen05 fence here
           const uint32_t a_addr = smem_u32(sA + stage * C::kATile);
           const uint32_t b_addr = smem_u32(sB + stage * C::kBTile);
 #pragma unroll
@@ -477,6 +481,422 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair version for 256-token tiles (tcgen05 cta_group::2).
+//
+// The two CTAs of a cluster share one tile of 256 weight rows x 256 tokens.
+// CTA r expands weight rows r*128.. of the tile into its own shared memory and
+// loads tokens r*128.. of the activation tile; one M = 256, N = 256 MMA issued
+// by the even CTA reads both halves of both operands, and each CTA's TMEM
+// receives the accumulator of its own 128 weight rows over all 256 tokens.
+// Per SM and K step this streams half the activation bytes of the single-CTA
+// kernel (16 KB instead of 32 KB), the L2-to-SM traffic that bounds that
+// kernel at 256 tokens, and halves the activation reads from shared memory.
+//
+// Barriers (E = the even CTA):
+//   tma_full[s]   in E: E's producer expects both CTAs' activation (and
+//                 extension) bytes; both CTAs' TMA loads complete on it
+//   codes_full[s] in each CTA: that CTA's code tile landed (local TMA); on an
+//                 extension step a plain arrival, so it has a phase per stage use
+//   deq_full[d]   in E: one arrival per dequantizer warp of both CTAs (8) per
+//                 main K step; its ring index d counts main steps only
+//   empty[s]      in each CTA: E's MMA completion, multicast (stage reusable)
+//   acc_full[a]   in each CTA: E's MMA completion, multicast (accumulator a)
+//   acc_empty[a]  in E: one arrival per epilogue warp of both CTAs (8)
+// ---------------------------------------------------------------------------
+template <int kStages, bool kBwd, int kGroups, int kNT>
+struct PCfg {
+  static constexpr int BN = 256;             // tokens per MMA (N), HALF of them in each CTA
+  static constexpr int HALF = 128;
+  // Token tiles of BN per unit: with 2, each expanded weight tile feeds two MMAs (512
+  // tokens), halving the expansion work per flop; the two accumulators then fill TMEM,
+  // so the epilogue of a unit is not overlapped with the next unit's MMAs.
+  static constexpr int NT = kNT;
+  static constexpr int TOK = BN * NT;
+  static constexpr int kAccSets = (kNT == 1) ? 2 : 1;
+  static constexpr int Stages = kStages;
+  static constexpr bool Bwd = kBwd;
+  static constexpr int kATile = 128 * 64 * 2;
+  static constexpr int kBTile = HALF * 64 * 2;
+  static constexpr int kRBytes = 4096;
+  // Dequantizer groups of four warps: group g expands the main K steps whose ring
+  // index is g modulo kGroups, so kGroups steps are in expansion at once.
+  static constexpr int Groups = kGroups;
+  static constexpr int kThreads = (6 + 4 * kGroups) * 32;
+  static constexpr int kTmemCols = 512;      // two accumulators of 256 columns
+  static constexpr int kBStage = NT * kBTile;  // activation bytes of one stage in one CTA
+  static constexpr int kSmemBytes = Stages * (kATile + kBStage + kRBytes) + 1024 + 256;
+  static_assert(kStages % kGroups == 0, "the ring index modulo kGroups picks the dequantizer group");
+  static_assert(kNT == 1 || kNT == 2, "one or two token tiles per unit");
+  static_assert(kAccSets * TOK <= kTmemCols, "TMEM columns");
+  static_assert(4 * kStages + 4 <= 31, "barrier area");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    qlora_wgemm_pair_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ WMaps maps) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);   // same offsets in both CTAs
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::Stages * C::kATile;
+  uint8_t* sR = sB + C::Stages * C::kBStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + C::Stages * C::kRBytes);
+  uint64_t* tma_full = bars;
+  uint64_t* codes_full = tma_full + C::Stages;
+  uint64_t* deq_full = codes_full + C::Stages;
+  uint64_t* empty = deq_full + C::Stages;
+  uint64_t* acc_full = empty + C::Stages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const bool even = (rank == 0);
+  const int pair = static_cast<int>(cluster_id_x());
+  const int pairs = static_cast<int>(cluster_count_x());
+  const int units = p.tiles_m * p.tiles_n * p.splits;     // tiles_m counts 256-row tiles
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::Stages; ++s) {
+      mbar_init(&tma_full[s], 1);
+      mbar_init(&codes_full[s], 1);
+      mbar_init(&deq_full[s], 8);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();      // both CTAs' barriers exist before any remote arrival or load lands on them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.act);
+      tma_prefetch_desc(&maps.codes);
+      tma_prefetch_desc(&maps.a2);
+      tma_prefetch_desc(&maps.b2);
+      int stage = 0;
+      uint32_t ph = 0;
+      uint32_t pend_codes = 0, pend_full = 0, pend_par = 0;
+      bool ok = true;
+      for (int u = pair; u < units && ok; u += pairs) {
+        int mb, nb, split, kt0, nmain, next;
+        wdecode(p, u, mb, nb, split, kt0, nmain, next);
+        const int mh = 2 * mb + rank;                      // this CTA's 128-row tile
+        const int tok0 = nb * C::TOK + rank * C::HALF;     // + t * BN for token tile t
+        for (int i = 0; i < nmain + next; ++i) {
+          if (!mbar_wait(&empty[stage], ph ^ 1)) { ok = false; break; }
+          pend_codes &= ~(1u << stage);
+          pend_full &= ~(1u << stage);
+          const uint32_t full_e = smem_cluster_addr(&tma_full[stage], 0);
+          uint8_t* a_dst = sA + stage * C::kATile;
+          uint8_t* b_dst = sB + stage * C::kBStage;
+          if (i < nmain) {
+            const int kt = kt0 + i;
+            mbar_arrive_expect_tx(&codes_full[stage], C::kRBytes);
+            if (C::Bwd) tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], mh * 64, kt * 64);
+            else tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], kt * 32, mh * 128);
+            pend_codes |= (1u << stage);
+            if (even) mbar_arrive_expect_tx(&tma_full[stage], 2 * C::kBStage);
+#pragma unroll
+            for (int t = 0; t < C::NT; ++t)
+              tma_load_2d_pair(b_dst + t * C::kBTile, &maps.act, full_e, kt * 64, tok0 + t * C::BN);
+          } else {
+            const int e = i - nmain;
+            // no codes for an extension step: complete codes_full's phase anyway, so that its
+            // phases count every use of the stage as the dequantizers' ring phase does
+            mbar_arrive(&codes_full[stage]);
+            if (even) mbar_arrive_expect_tx(&tma_full[stage], 2 * (C::kATile + C::kBStage));
+            if (C::Bwd) {
+              tma_load_2d_pair(a_dst, &maps.a2, full_e, mh * 128, e * 64);
+              tma_load_2d_pair(a_dst + 8192, &maps.a2, full_e, mh * 128 + 64, e * 64);
+            } else {
+              tma_load_2d_pair(a_dst, &maps.a2, full_e, e * 64, mh * 128);
+            }
+#pragma unroll
+            for (int t = 0; t < C::NT; ++t)
+              tma_load_2d_pair(b_dst + t * C::kBTile, &maps.b2, full_e, e * 64, tok0 + t * C::BN);
+          }
+          pend_full |= (1u << stage);
+          pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
+          if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+        }
+      }
+      if (ok) {
+        for (int s = 0; s < C::Stages; ++s) {   // every stage released once more: no load still lands
+          if (!mbar_wait(&empty[stage], ph ^ 1)) break;
+          if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+        }
+      } else {
+        for (int s = 0; s < C::Stages; ++s) {
+          if (pend_codes & (1u << s)) mbar_wait(&codes_full[s], (pend_par >> s) & 1u);
+          if (even && (pend_full & (1u << s))) mbar_wait(&tma_full[s], (pend_par >> s) & 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (even && lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(C::BN, C::Bwd, false, 256);
+      // Descriptors: fixed fields once; per stage only the start address (16-byte units)
+      // changes, and a K step of 16 moves it by 32 bytes (K-major) or 2048 bytes (MN-major).
+      const uint64_t a_desc0 = C::Bwd ? umma_desc_sw128(smem_u32(sA), 8192, 1024) : umma_desc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
+      constexpr uint64_t kAStep = C::Bwd ? (2048 >> 4) : (32 >> 4);
+      constexpr uint64_t kBStep = 32 >> 4;
+      int stage = 0, dstage = 0, acc = 0;
+      uint32_t ph = 0, dph = 0, aph = 0;
+      bool ok = true;
+      for (int u = pair; u < units && ok; u += pairs) {
+        int mb, nb, split, kt0, nmain, next;
+        wdecode(p, u, mb, nb, split, kt0, nmain, next);
+        if (!mbar_wait(&acc_empty[acc], aph ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::TOK);
+        for (int i = 0; i < nmain + next; ++i) {
+          if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
+          if (i < nmain) {
+            if (!mbar_wait(&deq_full[dstage], dph)) { ok = false; break; }
+            if (++dstage == C::Stages) { dstage = 0; dph ^= 1; }
+          }
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>(stage) * (C::kATile >> 4);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(stage) * (C::kBStage >> 4);
+#pragma unroll
+          for (int t = 0; t < C::NT; ++t) {
+            const uint32_t dt = d_tmem + static_cast<uint32_t>(t * C::BN);
+            const uint64_t bt = bd + static_cast<uint64_t>(t) * (C::kBTile >> 4);
+            umma_bf16_pair(dt, ad, bt, idesc, i > 0 ? 1u : 0u);
+            umma_bf16_pair(dt, ad + kAStep, bt + kBStep, idesc, 1u);
+            umma_bf16_pair(dt, ad + 2 * kAStep, bt + 2 * kBStep, idesc, 1u);
+            umma_bf16_pair(dt, ad + 3 * kAStep, bt + 3 * kBStep, idesc, 1u);
+          }
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&acc_full[acc], 0x3);
+        if (++acc == C::kAccSets) { acc = 0; aph ^= 1; }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t acc_empty_e0 = smem_cluster_addr(&acc_empty[0], 0);
+    const uint32_t acc_empty_e1 = smem_cluster_addr(&acc_empty[1], 0);
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = pair; u < units; u += pairs) {
+      int mb, nb, split, kt0, nmain, next;
+      wdecode(p, u, mb, nb, split, kt0, nmain, next);
+      if (!mbar_wait(&acc_full[acc], aph)) break;
+      tc_fence_after();
+      const int feat = (2 * mb + rank) * 128 + q * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::TOK);
+#pragma unroll 1
+      for (int c = 0; c < C::TOK / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, v);
+        tmem_ld_wait();
+        wstore<32>(p, split, feat, nb * C::TOK + c * 32, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc ? acc_empty_e1 : acc_empty_e0);
+      if (++acc == C::kAccSets) { acc = 0; aph ^= 1; }
+    }
+  } else {
+    // ------------------------------------------------------------ dequantizers (both CTAs)
+    // As in the single-CTA kernel, on this CTA's 128-row tile, with C::Groups groups taking
+    // main K steps in turn; each warp reports its finished tile to the even CTA's deq_full.
+    const int grp = (warp - 6) >> 2;
+    const int gt = threadIdx.x - 192 - 128 * grp;    // 0..127
+    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
+    const int i_mn = gt & 63;
+    const int c_mn = gt >> 6;
+    uint32_t r_off0, r_off1, a_off;
+    int sw;
+    if (!C::Bwd) {
+      const uint32_t x = (gt >> 2) & 1;                         // 32B swizzle of the code tile
+      r_off0 = gt * 32 + 16 * x;
+      r_off1 = gt * 32 + 16 * (x ^ 1);
+      a_off = (gt >> 3) * 1024 + (gt & 7) * 128;
+      sw = gt & 7;
+    } else {
+      const uint32_t x = (i_mn >> 1) & 3;                       // 64B swizzle of the code tile
+      r_off0 = i_mn * 64 + 16 * ((2 * c_mn) ^ x);
+      r_off1 = i_mn * 64 + 16 * ((2 * c_mn + 1) ^ x);
+      a_off = c_mn * 8192 + (i_mn >> 3) * 1024 + (i_mn & 7) * 128;
+      sw = i_mn & 7;
+    }
+    const uint32_t deq_e = smem_cluster_addr(deq_full, 0);    // deq_full[d] of the even CTA: deq_e + 8 d
+    int stage = 0, dstage = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = pair; u < units && ok; u += pairs) {
+      int mb, nb, split, kt0, nmain, next;
+      wdecode(p, u, mb, nb, split, kt0, nmain, next);
+      const int mh = 2 * mb + rank;
+      const int first = (grp - dstage % C::Groups + C::Groups) % C::Groups;   // first own main step
+      constexpr int G = C::Groups;
+      auto block_of = [&](int i, bool& valid) -> int64_t {
+        const int kt = kt0 + i;
+        int64_t wrow, kb;
+        if (!C::Bwd) { wrow = static_cast<int64_t>(mh) * 128 + gt; kb = kt; }
+        else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(mh) * 2 + c_mn; }
+        valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
+        return wrow * p.w_kblocks + kb;
+      };
+      RawScale r0{0u, 0.f}, r1{0u, 0.f}, r2{0u, 0.f}, r3{0u, 0.f};
+      {
+        bool v;
+        int64_t bb = block_of(first, v);
+        if (first < nmain && v) r0 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + G, v);
+        if (first + G < nmain && v) r1 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 2 * G, v);
+        if (first + 2 * G < nmain && v) r2 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 3 * G, v);
+        if (first + 3 * G < nmain && v) r3 = load_raw_scale(p.scales, bb);
+      }
+      for (int i = 0; i < nmain + next; ++i) {
+        if (i < nmain) {
+          if (dstage % G == grp) {
+            bool valid, v4;
+            block_of(i, valid);
+            const int64_t b4 = block_of(i + 4 * G, v4);
+            RawScale r4{0u, 0.f};
+            if (i + 4 * G < nmain && v4) r4 = load_raw_scale(p.scales, b4);
+            if (!mbar_wait(&codes_full[stage], ph)) { ok = false; break; }
+            const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
+            if (valid) {
+              const uint32_t rsrc = smem_u32(sR + stage * C::kRBytes);
+              const uint4 w0 = ld_shared_v4_w(rsrc + r_off0);
+              const uint4 w1 = ld_shared_v4_w(rsrc + r_off1);
+              const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales, r0, mean));
+              st_shared_v4_w(adst + ((0 ^ sw) << 4), nf4_lookup8(lut, w0.x));
+              st_shared_v4_w(adst + ((1 ^ sw) << 4), nf4_lookup8(lut, w0.y));
+              st_shared_v4_w(adst + ((2 ^ sw) << 4), nf4_lookup8(lut, w0.z));
+              st_shared_v4_w(adst + ((3 ^ sw) << 4), nf4_lookup8(lut, w0.w));
+              st_shared_v4_w(adst + ((4 ^ sw) << 4), nf4_lookup8(lut, w1.x));
+              st_shared_v4_w(adst + ((5 ^ sw) << 4), nf4_lookup8(lut, w1.y));
+              st_shared_v4_w(adst + ((6 ^ sw) << 4), nf4_lookup8(lut, w1.z));
+              st_shared_v4_w(adst + ((7 ^ sw) << 4), nf4_lookup8(lut, w1.w));
+            } else {
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) st_shared_v4_w(adst + (j << 4), z);
+            }
+            // expanded tile visible to the async proxy (either SM's tensor core reads it);
+            // code reads ordered before the slot's async refill
+            fence_proxy_async_smem();
+            r0 = r1;
+            r1 = r2;
+            r2 = r3;
+            r3 = r4;
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(deq_e + static_cast<uint32_t>(dstage) * 8u);
+          }
+          if (++dstage == C::Stages) dstage = 0;
+        }
+        if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();      // no CTA leaves while the other may still arrive on its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
+template <class C>
+static cudaError_t launch_pcfg(const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(qlora_wgemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
+  if (grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qlora_wgemm_pair_kernel<C>, p, maps);
+}
+
+// CTA pairs of the 256-token kernel that fit on the device at once (one CTA per SM).
+int wgemm_pair_slots() {
+  static int cached[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 74;   // no device: a B200's 148 SMs
+  std::lock_guard<std::mutex> g(mu);
+  if (cached[dev] > 0) return cached[dev];
+  using C = PCfg<6, false, 2, 1>;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+  int slots = sms / 2;
+  if (cudaFuncSetAttribute(qlora_wgemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes) == cudaSuccess) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, qlora_wgemm_pair_kernel<C>, &cfg) == cudaSuccess && n > 0 && n < slots)
+      slots = n;
+  }
+  cudaGetLastError();
+  cached[dev] = slots > 0 ? slots : 1;
+  return cached[dev];
+}
+
 template <class C>
 static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
@@ -497,13 +917,22 @@ static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid,
   return cudaGetLastError();
 }
 
-int wgemm_box_rows(int bn) { return bn == 384 ? 192 : bn; }
+int wgemm_box_rows(int bn) { return bn >= 256 ? 128 : bn; }   // a CTA pair loads half of each 256-token tile
+
+int wgemm_tile_rows(int bn) { return bn >= 256 ? 256 : 128; }  // weight rows per tile (two CTAs from 256 tokens)
+
+int wgemm_grid(const GemmParams& p, int bn, int sms) {
+  const int64_t units = static_cast<int64_t>(p.tiles_m) * p.tiles_n * p.splits;
+  if (bn >= 256) return static_cast<int>(2 * std::min<int64_t>(units, wgemm_pair_slots()));
+  return static_cast<int>(std::min<int64_t>(units, sms));
+}
 
 int wgemm_bn(int64_t tokens) {
   if (tokens <= 16) return 16;
   if (tokens <= 64) return 64;
   if (tokens <= 128) return 128;
-  return 256;
+  if (tokens <= kPair512From) return 256;
+  return 512;
 }
 
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
@@ -516,14 +945,16 @@ cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& map
       case 16: e = launch_wcfg<WCfg<16, 1, 8, false>>(p, maps, grid, st); break;
       case 64: e = launch_wcfg<WCfg<64, 1, 8, false>>(p, maps, grid, st); break;
       case 128: e = launch_wcfg<WCfg<128, 1, 6, false>>(p, maps, grid, st); break;
-      case 256: e = launch_wcfg<WCfg<256, 1, 4, false>>(p, maps, grid, st); break;
+      case 256: e = launch_pcfg<PCfg<6, false, 2, 1>>(p, maps, grid, st); break;   // CTA pair
+      case 512: e = launch_pcfg<PCfg<4, false, 2, 2>>(p, maps, grid, st); break;   // CTA pair, two token tiles
     }
   } else {
     switch (bn) {
       case 16: e = launch_wcfg<WCfg<16, 1, 8, true>>(p, maps, grid, st); break;
       case 64: e = launch_wcfg<WCfg<64, 1, 8, true>>(p, maps, grid, st); break;
       case 128: e = launch_wcfg<WCfg<128, 1, 6, true>>(p, maps, grid, st); break;
-      case 256: e = launch_wcfg<WCfg<256, 1, 4, true>>(p, maps, grid, st); break;
+      case 256: e = launch_pcfg<PCfg<6, true, 2, 1>>(p, maps, grid, st); break;    // CTA pair
+      case 512: e = launch_pcfg<PCfg<4, true, 2, 2>>(p, maps, grid, st); break;    // CTA pair, two token tiles
     }
   }
   if (timed) timing_record(st, false, algo_flops);

@@ -228,10 +228,12 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   P.da = choose_split(cdiv(k, 128), cdiv(m, 64), sms);
   P.bn = wgemm_bn(m);
   const int64_t tok_tiles = cdiv(m, P.bn);
-  const int64_t fwd_tiles = cdiv(n, 128) * tok_tiles;
-  P.fwd = choose_wsplit(fwd_tiles, k / 64, sms, m * n);
-  const int64_t bwd_tiles = cdiv(k, 128) * tok_tiles;
-  P.bwd = choose_wsplit(bwd_tiles, cdiv(n, 64), sms, m * k);
+  const int64_t wrows = wgemm_tile_rows(P.bn);
+  const int wslots = (wrows == 256) ? wgemm_pair_slots() : sms;   // a CTA pair works one 256-row tile
+  const int64_t fwd_tiles = cdiv(n, wrows) * tok_tiles;
+  P.fwd = choose_wsplit(fwd_tiles, k / 64, wslots, m * n);
+  const int64_t bwd_tiles = cdiv(k, wrows) * tok_tiles;
+  P.bwd = choose_wsplit(bwd_tiles, cdiv(n, 64), wslots, m * k);
   const size_t rp = static_cast<size_t>(P.r_pad);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -543,6 +545,7 @@ int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m,
 
   // Y^T = W . X^T + B . (sU)^T with W dequantized on the fly (weight as the 128-row operand)
   GemmParams p = base_params(n, m, P.bn, k / 64, P.fwd);
+  p.tiles_m = static_cast<int32_t>(cdiv(n, wgemm_tile_rows(P.bn)));
   p.ext_tiles = P.r_pad / 64;
   p.scales = scale_src(w);
   p.w_kblocks = k / 64;
@@ -565,7 +568,7 @@ int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m,
   ok = ok && map_bf16(&maps.b2, sU, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
   if (!ok) return QLORA_ERR_CUDA;
   const double fwd_flops = 2.0 * double(m) * double(n) * double(k + r);
-  cudaError_t e = launch_wgemm(false, P.bn, p, maps, grid_of(p), st, fwd_flops);
+  cudaError_t e = launch_wgemm(false, P.bn, p, maps, wgemm_grid(p, P.bn, num_sms()), st, fwd_flops);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   if (P.fwd.splits > 1) {
     e = launch_splitk_reduce(static_cast<const float*>(p.out), P.fwd.splits, p.part_stride, m, n, n, Y,
@@ -631,6 +634,7 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
   if (dX != nullptr) {
     // dX^T = W^T . dY^T + A^T . (sG)^T, W dequantized into the MN-major operand layout
     GemmParams p = base_params(k, m, P.bn, cdiv(n, 64), P.bwd);
+    p.tiles_m = static_cast<int32_t>(cdiv(k, wgemm_tile_rows(P.bn)));
     p.ext_tiles = D.on ? 0 : P.r_pad / 64;     // under dropout the low-rank term is added masked, below
     p.scales = scale_src(w);
     p.w_kblocks = k / 64;
@@ -655,7 +659,8 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
     ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
     if (!ok) return QLORA_ERR_CUDA;
     const double dx_flops = 2.0 * double(m) * double(k) * double(n + r);
-    if (launch_wgemm(true, P.bn, p, maps, grid_of(p), st, dx_flops) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_wgemm(true, P.bn, p, maps, wgemm_grid(p, P.bn, num_sms()), st, dx_flops) != cudaSuccess)
+      return QLORA_ERR_CUDA;
     if (P.bwd.splits > 1 &&
         launch_splitk_reduce(static_cast<const float*>(p.out), P.bwd.splits, p.part_stride, m, k, k, dX,
                              dx_dtype == QLORA_DTYPE_BF16, acc_dx, st) != cudaSuccess)

@@ -117,7 +117,10 @@ struct WMaps {
   CUtensorMap b2;      // low-rank B-side tile: s*U or s*G [tokens, r_pad]
 };
 int wgemm_bn(int64_t tokens);          // tokens per tile
-int wgemm_box_rows(int bn);              // token rows per TMA box / MMA (the tile may hold two)
+int wgemm_box_rows(int bn);              // token rows per TMA box (each CTA of a pair loads half)
+int wgemm_tile_rows(int bn);             // weight rows per tile: 256 when a CTA pair shares it
+int wgemm_pair_slots();                  // CTA pairs resident at once
+int wgemm_grid(const GemmParams& p, int bn, int sms);   // CTAs to launch (even for CTA pairs)
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
                          double algo_flops);
 
