@@ -33,7 +33,7 @@ EXPORTED = (
     "qlora_nf4_quantize_workspace_bytes", "qlora_nf4_quantize", "qlora_nf4_dequantize",
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_silu_gate_fwd", "qlora_silu_gate_bwd", "qlora_check_device_error",
-    "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end",
+    "qlora_launch_count", "qlora_timing_begin", "qlora_timing_end", "qlora_timing_launch",
     "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
     "qlora_adamw_step", "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch",
@@ -116,6 +116,7 @@ def lib() -> ctypes.CDLL:
         "qlora_launch_count": (ctypes.c_int64, []),
         "qlora_timing_begin": (ctypes.c_int, [i32]),
         "qlora_timing_end": (ctypes.c_int, [vp, vp, vp]),
+        "qlora_timing_launch": (ctypes.c_int, [i32, vp, vp]),
         "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
         "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
@@ -345,6 +346,16 @@ def qlora_timing_end():
     _check(lib().qlora_timing_end(ctypes.addressof(ms), ctypes.addressof(n), ctypes.addressof(fl)),
            "qlora_timing_end")
     return ms.value, n.value, fl.value
+
+
+def qlora_timing_launches(count: int):
+    """Per-launch (device ms, algorithmic flops) of the last qlora_timing_end, in launch order."""
+    out = []
+    for i in range(int(count)):
+        ms, fl = ctypes.c_double(0), ctypes.c_double(0)
+        _check(lib().qlora_timing_launch(i, ctypes.addressof(ms), ctypes.addressof(fl)), "qlora_timing_launch")
+        out.append((ms.value, fl.value))
+    return out
 
 
 def qlora_nf4_quantize_noalloc(W: torch.Tensor, w: QuantizedWeight, stream=None):

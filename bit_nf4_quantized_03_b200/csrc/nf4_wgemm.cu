@@ -98,12 +98,43 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-// Raw scale of one block, loaded ahead of use; turned into the fp32 scale later.
-// Epilogue: 32 (or 16) consecutive tokens of one output feature.
+// Epilogue: 32 (or 16) consecutive tokens of one output feature. When accumulating,
+// every old value of the chunk is read before any is written back, so the chunk
+// costs one memory round trip (a load after each store could not be reordered: the
+// compiler cannot prove the addresses distinct).
 template <int kCount>
 __device__ __forceinline__ void wstore(const GemmParams& p, int split, int feat, int tok0, const uint32_t (&v)[32]) {
   if (feat >= p.rows) return;
   const int64_t ld = p.ld_out;
+  const int nvalid = p.cols - tok0;     // tokens of the chunk inside the output (may be < kCount or <= 0)
+  if (p.accumulate && p.out_mode != kOutPartial) {
+    constexpr int kBatch = (kCount == 32) ? 32 : 8;   // smaller batches keep the 16-token kernel unspilled
+#pragma unroll
+    for (int j0 = 0; j0 < kCount; j0 += kBatch) {
+      float old[kBatch];
+#pragma unroll
+      for (int jj = 0; jj < kBatch; ++jj) {
+        const int j = j0 + jj;
+        old[jj] = 0.f;
+        if (j < nvalid) {
+          const int64_t off = static_cast<int64_t>(tok0 + j) * ld + feat;
+          if (p.out_mode == kOutF32) old[jj] = static_cast<const float*>(p.out)[off];
+          else old[jj] = __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p.out)[off]) << 16);
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < kBatch; ++jj) {
+        const int j = j0 + jj;
+        if (j < nvalid) {
+          const int64_t off = static_cast<int64_t>(tok0 + j) * ld + feat;
+          const float y = __uint_as_float(v[j]) + old[jj];
+          if (p.out_mode == kOutF32) static_cast<float*>(p.out)[off] = y;
+          else static_cast<uint16_t*>(p.out)[off] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+        }
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < kCount; ++j) {
     const int m = tok0 + j;
@@ -113,12 +144,9 @@ __device__ __forceinline__ void wstore(const GemmParams& p, int split, int feat,
     if (p.out_mode == kOutPartial) {
       static_cast<float*>(p.out)[split * p.part_stride + off] = x;
     } else if (p.out_mode == kOutF32) {
-      float* o = static_cast<float*>(p.out) + off;
-      *o = p.accumulate ? (*o + x) : x;
+      static_cast<float*>(p.out)[off] = x;
     } else {
-      uint16_t* o = static_cast<uint16_t*>(p.out) + off;
-      const float y = p.accumulate ? (x + __uint_as_float(static_cast<uint32_t>(*o) << 16)) : x;
-      *o = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+      static_cast<uint16_t*>(p.out)[off] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
     }
   }
 }
@@ -937,6 +965,10 @@ int wgemm_bn(int64_t tokens) {
 
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
                          double algo_flops) {
+  // the tile counts must be those of the kernel this width selects
+  if (p.tiles_n != (static_cast<int64_t>(p.cols) + bn - 1) / bn ||
+      p.tiles_m != (static_cast<int64_t>(p.rows) + wgemm_tile_rows(bn) - 1) / wgemm_tile_rows(bn))
+    return cudaErrorInvalidValue;
   const bool timed = timing_active();
   if (timed) timing_record(st, true, algo_flops);
   cudaError_t e = cudaErrorInvalidValue;

@@ -23,6 +23,7 @@ std::mutex g_timing_mu;
 std::vector<cudaEvent_t> g_events;     // pairs: start, stop
 std::vector<double> g_event_flops;
 size_t g_events_used = 0;
+std::vector<double> g_last_ms, g_last_flops;   // per launch, from the last qlora_timing_end
 }  // namespace
 
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -254,7 +255,9 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   part = std::max(part, static_cast<size_t>(P.da.splits) * k * rp);
   if (P.fwd.splits > 1) part = std::max(part, static_cast<size_t>(P.fwd.splits) * m * n);
   if (m <= 64) part = std::max(part, static_cast<size_t>(lora_down_small_slices(k)) * m * rp);
-  if (P.bwd.splits > 1) part = std::max(part, static_cast<size_t>(P.bwd.splits) * m * k);
+  // dX through fp32 partials: for split K, and for an accumulating dX on the CTA-pair path
+  if (P.bwd.splits > 1 || wrows == 256)
+    part = std::max(part, static_cast<size_t>(std::max(P.bwd.splits, 1)) * m * k);
   P.off_part = take(part * 4);
   P.total = off;
   return P;
@@ -633,15 +636,21 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
 
   if (dX != nullptr) {
     // dX^T = W^T . dY^T + A^T . (sG)^T, W dequantized into the MN-major operand layout
-    GemmParams p = base_params(k, m, P.bn, cdiv(n, 64), P.bwd);
-    p.tiles_m = static_cast<int32_t>(cdiv(k, wgemm_tile_rows(P.bn)));
+    const int acc_dx = (flags & QLORA_BWD_ACCUMULATE_DX) ? 1 : 0;
+    const int bn = P.bn;
+    const Split& sp = P.bwd;
+    // Accumulating on the CTA-pair path goes through fp32 partials and the reduce pass: in the
+    // GEMM's epilogue the old dX values (rows ld apart) were read at a small fraction of the
+    // memory's speed and stalled the tensor cores; the streaming reduce reads them coalesced.
+    const bool via_part = sp.splits > 1 || (acc_dx && wgemm_tile_rows(bn) == 256);
+    GemmParams p = base_params(k, m, bn, cdiv(n, 64), sp);
+    p.tiles_m = static_cast<int32_t>(cdiv(k, wgemm_tile_rows(bn)));
     p.ext_tiles = D.on ? 0 : P.r_pad / 64;     // under dropout the low-rank term is added masked, below
     p.scales = scale_src(w);
     p.w_kblocks = k / 64;
     p.w_rows = static_cast<int32_t>(n);
     p.ld_out = k;
-    const int acc_dx = (flags & QLORA_BWD_ACCUMULATE_DX) ? 1 : 0;
-    if (P.bwd.splits > 1) {
+    if (via_part) {
       p.out = wsb + P.off_part;
       p.part_stride = m * k;
       p.out_mode = kOutPartial;
@@ -652,17 +661,17 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
     }
     WMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    bool ok = map_bf16(&maps.act, dY, m, n, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
+    bool ok = map_bf16(&maps.act, dY, m, n, static_cast<uint32_t>(wgemm_box_rows(bn)));
     ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
                        static_cast<uint64_t>(k / 2), 64, 64, 64);
     ok = ok && tmap_2d(&maps.a2, A, kBF16, k, r, k * 2, 64, 64, 128);
-    ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
+    ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(bn)));
     if (!ok) return QLORA_ERR_CUDA;
     const double dx_flops = 2.0 * double(m) * double(k) * double(n + r);
-    if (launch_wgemm(true, P.bn, p, maps, wgemm_grid(p, P.bn, num_sms()), st, dx_flops) != cudaSuccess)
+    if (launch_wgemm(true, bn, p, maps, wgemm_grid(p, bn, num_sms()), st, dx_flops) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    if (P.bwd.splits > 1 &&
-        launch_splitk_reduce(static_cast<const float*>(p.out), P.bwd.splits, p.part_stride, m, k, k, dX,
+    if (via_part &&
+        launch_splitk_reduce(static_cast<const float*>(p.out), p.splits, p.part_stride, m, k, k, dX,
                              dx_dtype == QLORA_DTYPE_BF16, acc_dx, st) != cudaSuccess)
       return QLORA_ERR_CUDA;
     if (D.on) {
@@ -762,6 +771,8 @@ int qlora_timing_end(double* total_ms, int32_t* launches, double* flops) {
   qlora::g_timing_on = false;
   double ms = 0.0, fl = 0.0;
   int rc = QLORA_OK;
+  qlora::g_last_ms.clear();
+  qlora::g_last_flops.clear();
   for (size_t i = 0; i + 1 < qlora::g_events_used; i += 2) {
     float t = 0.f;
     if (cudaEventSynchronize(qlora::g_events[i + 1]) != cudaSuccess ||
@@ -771,6 +782,8 @@ int qlora_timing_end(double* total_ms, int32_t* launches, double* flops) {
     }
     ms += t;
     fl += qlora::g_event_flops[i / 2];
+    qlora::g_last_ms.push_back(t);
+    qlora::g_last_flops.push_back(qlora::g_event_flops[i / 2]);
   }
   if (total_ms) *total_ms = ms;
   if (launches) *launches = static_cast<int32_t>(qlora::g_events_used / 2);
@@ -780,6 +793,15 @@ int qlora_timing_end(double* total_ms, int32_t* launches, double* flops) {
   qlora::g_event_flops.clear();
   qlora::g_events_used = 0;
   return rc;
+}
+
+int qlora_timing_launch(int32_t index, double* ms, double* flops) {
+  std::lock_guard<std::mutex> g(qlora::g_timing_mu);
+  if (index < 0 || static_cast<size_t>(index) >= qlora::g_last_ms.size() || ms == nullptr || flops == nullptr)
+    return QLORA_ERR_INVALID;
+  *ms = qlora::g_last_ms[static_cast<size_t>(index)];
+  *flops = qlora::g_last_flops[static_cast<size_t>(index)];
+  return QLORA_OK;
 }
 
 int qlora_selftest_wait_timeout(int32_t limit_ms, qlora_stream_t stream) {

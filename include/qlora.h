@@ -313,6 +313,11 @@ int64_t qlora_launch_count(void);
 int qlora_timing_begin(int32_t max_launches);
 int qlora_timing_end(double *total_ms, int32_t *launches, double *flops);
 
+/* Device time (ms) and algorithmic flops of launch `index` (0-based, launch
+ * order) of the last qlora_timing_end. QLORA_ERR_INVALID for an index outside
+ * [0, launches) or a null pointer. Process-wide, not thread-safe. */
+int qlora_timing_launch(int32_t index, double *ms, double *flops);
+
 /* Exercises the failure path without faulting the GPU: launches one thread
  * that waits on a barrier nobody arrives on and gives up after limit_ms
  * (1..2000), recording the device error word exactly as a stuck pipeline

@@ -36,6 +36,14 @@ def test_library_exports_every_declared_symbol(L):
     assert sorted(q.EXPORTED) == syms
 
 
+def test_timing_launch_rejects_indexes_without_a_record(L):
+    # host bookkeeping only: before any timed launch there is no record to read (1 = QLORA_ERR_INVALID)
+    ms, fl = ctypes.c_double(0), ctypes.c_double(0)
+    assert L.qlora_timing_launch(0, ctypes.addressof(ms), ctypes.addressof(fl)) == 1
+    assert L.qlora_timing_launch(-1, ctypes.addressof(ms), ctypes.addressof(fl)) == 1
+    assert L.qlora_timing_launch(0, None, None) == 1
+
+
 def test_host_level_table_matches_oracle_bitwise(L):
     lv, mid = q.qlora_nf4_levels()
     lv = np.array(lv, dtype=np.float32)

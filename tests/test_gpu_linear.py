@@ -76,6 +76,26 @@ def test_accumulate_flags():
     check_close(dB.cpu(), dB_ref + dB0.double().numpy(), "dB+")
 
 
+@pytest.mark.parametrize("dx_dtype", [q.QLORA_DTYPE_FP32, q.QLORA_DTYPE_BF16])
+def test_accumulate_dx_many_tokens(dx_dtype):
+    # on the CTA-pair path an accumulating dX goes through fp32 partials and the reduce pass while a
+    # plain one is written by the GEMM: both against the oracle, on ragged token and feature counts
+    L = Layer(2312, 520, 1088, 16)
+    Wd = L.oracle_weight()
+    dX_ref, _, _ = o.linear_backward(Wd, L.X, L.dY, L.A, L.B, L.alpha)
+    g = torch.Generator().manual_seed(7)
+    dX0 = torch.randn(L.m, L.k, generator=g)
+    if dx_dtype == q.QLORA_DTYPE_BF16:
+        dX0 = dX0.to(torch.bfloat16).float()
+        dX = dX0.to(torch.bfloat16).cuda()
+    else:
+        dX = dX0.clone().cuda()
+    L.bwd(None, dx_dtype, q.QLORA_BWD_ACCUMULATE_DX, dX)
+    check_close(dX.float().cpu(), dX_ref + dX0.double().numpy(), "dX+", bf16_out=(dx_dtype == q.QLORA_DTYPE_BF16))
+    dXp, _, _ = L.bwd(None, dx_dtype)
+    check_close(dXp.float().cpu(), dX_ref, "dX", bf16_out=(dx_dtype == q.QLORA_DTYPE_BF16))
+
+
 def test_backward_without_dx():
     L = Layer(128, 256, 256, 8)
     Wd = L.oracle_weight()
