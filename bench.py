@@ -50,8 +50,8 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum; summary in
 # profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
 # recorded with it; any change to them prints null until the counters are taken again.
-WGEMM_TRAFFIC = {"bytes_per_launch": 954247497,
-                 "sources_sha256": "e5cae818f208f0d520cdde397fbf302ea5d0eafb114b8bd232e62c23205f3986"}
+WGEMM_TRAFFIC = {"bytes_per_launch": 910676891,
+                 "sources_sha256": "395e3aac4dca070a4dd98d35bd98389747527a92fc9972e376690d764b9899f9"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 

@@ -1,4 +1,4 @@
-// Fused NF4 GEMM with the frozen weight as the 128-row tensor-core operand.
+// Fused NF4 GEMM with the frozen weight as the tensor-core M operand.
 //
 //   forward   Y^T[n, m]  = W[n, :] . X[m, :]^T      + B[n, :] . (s U)[m, :]^T
 //   backward dX^T[k, m]  = W[:, k]^T . dY[m, :]^T   + A[:, k]^T . (s G)[m, :]^T
@@ -7,19 +7,24 @@
 // GPU multiplies", "QLoRA: Quantized Low-Rank Adaptation", Piece 2 and
 // "Batched 4-bit matmuls") straight into the 128-byte-swizzled shared-memory
 // tile that the tcgen05.mma descriptor reads, and is then reused by every
-// token of the tile: one MMA covers up to 256 tokens (its N), and for long
-// token counts two MMAs (two TMEM accumulators of 192 columns) share the same
-// weight tile, so each dequantized weight serves 384 tokens. Putting W on the
-// 128-row side is what makes this reuse possible, and at a handful of tokens
-// (M = 16) it wastes no tensor-core rows on padding.
+// token of the tile. Putting W on the M side is what makes this reuse
+// possible, and at a handful of tokens (M = 16) it wastes no tensor-core rows
+// on padding. Two kernels:
+//   qlora_wgemm_kernel       one CTA per 128-row weight tile, 16 to 128 tokens
+//                            per tile (MMA N), split K at few tokens
+//   qlora_wgemm_pair_kernel  above 128 tokens: two CTAs (a cluster on two SMs)
+//                            share a 256-row tile through tcgen05 cta_group::2;
+//                            above 1024 tokens each expanded weight tile feeds
+//                            two 256-token MMAs (512 tokens per unit), which
+//                            halves the expansion work per flop
 //
 // Warp roles (448 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA: packed codes (32B/64B-swizzled so the reads below are
 //               bank-conflict free), activation tiles, low-rank extension tiles
 //   warp 1      TMEM allocation + single-thread tcgen05.mma issue
 //   warps 2-5   epilogue: TMEM -> registers -> global (row-major Y / dX)
-//   warps 6-13  dequantizers: two lanes per weight row (32 codes each) expand
-//               every K step of the 128-row tile
+//   warps 6-13  dequantizers: two groups of four warps take turns on the K
+//               steps; one thread expands one row's 64-block per step
 #include <cudaTypedefs.h>
 
 #include <cstring>

@@ -182,7 +182,9 @@ int qlora_lora_merge(const qlora_nf4_weight *w, const uint16_t *A, const uint16_
                      void *W_out, int32_t out_dtype, qlora_stream_t stream);
 
 /* Bytes of device workspace qlora_linear_fwd / qlora_linear_bwd need for m
- * tokens, an [n, k] weight and rank r. */
+ * tokens, an [n, k] weight and rank r. Above 128 tokens this includes an fp32
+ * [m, k] buffer: a backward that accumulates into dX writes the GEMM's result
+ * there and adds it to dX in one coalesced pass. */
 size_t qlora_linear_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t r);
 
 /*
