@@ -433,8 +433,34 @@ def graph_time(fn, iters, flush) -> float:
     return max(replay_ms(g_op) - replay_ms(g_flush), 1e-6) / iters
 
 
+def _quant_components(q, synth, torch, dev, flush, peaks, out, qn, qk, sfx):
+    """Quantize (plain and double quant) and dequantize of one [qn, qk] weight with outliers."""
+    W = synth.weight(qn, qk, outlier_frac=0.001).to(dev)
+    ne = W.numel()
+    for mode, tag in ((q.QLORA_SCALE_BF16, "bf16"), (q.QLORA_SCALE_DQ_FP8, "dq_fp8")):
+        qw = q.QuantizedWeight(qn, qk, mode, device=dev)
+        ws = torch.empty(max(1, q.qlora_nf4_quantize_workspace_bytes(qn, qk, mode)), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda: q.qlora_nf4_quantize(W, qw, ws)
+        for _ in range(3):
+            fn()
+        ms = graph_time(fn, 20, flush)
+        scale_b = 2.0 / 64 if mode == q.QLORA_SCALE_BF16 else 1.0 / 64 + 4.0 / 16384
+        algo = ne * (4.0 + 0.5 + scale_b)
+        out[f"quantize_{tag}{sfx}"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6,
+                                       "frac": algo / ms / 1e6 / peaks["hbm_gbs"], "algo_bytes": algo}
+        o_ = torch.empty(qn, qk, dtype=torch.bfloat16, device=dev)
+        fn = lambda: q.qlora_nf4_dequantize(qw, o_)
+        for _ in range(3):
+            fn()
+        ms = graph_time(fn, 20, flush)
+        algo = ne * (0.5 + scale_b + 2.0)
+        out[f"dequantize_{tag}{sfx}"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6,
+                                         "frac": algo / ms / 1e6 / peaks["hbm_gbs"], "algo_bytes": algo}
+
+
 def components(dev, peaks) -> dict:
-    """Quantize / dequantize (4096 x 4096 with outliers) and M = 16 forward of
+    """Quantize / dequantize (4096 x 4096 and 22016 x 8192, with outliers) and M = 16 forward of
     the 65B q_proj, each against the measured HBM copy bandwidth. Timed by
     CUDA-graph replay so per-call host work (binding, tensor-map encoding)
     does not count; L2 is flushed before every call."""
@@ -443,28 +469,8 @@ def components(dev, peaks) -> dict:
     from bit_nf4_quantized_03_b200 import synth
     out = {}
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    W = synth.weight(4096, 4096, outlier_frac=0.001).to(dev)
-    ne = W.numel()
-    for mode, tag in ((q.QLORA_SCALE_BF16, "bf16"), (q.QLORA_SCALE_DQ_FP8, "dq_fp8")):
-        qw = q.QuantizedWeight(4096, 4096, mode, device=dev)
-        ws = torch.empty(max(1, q.qlora_nf4_quantize_workspace_bytes(4096, 4096, mode)), dtype=torch.uint8,
-                         device=dev)
-        fn = lambda: q.qlora_nf4_quantize(W, qw, ws)
-        for _ in range(3):
-            fn()
-        ms = graph_time(fn, 20, flush)
-        scale_b = 2.0 / 64 if mode == q.QLORA_SCALE_BF16 else 1.0 / 64 + 4.0 / 16384
-        algo = ne * (4.0 + 0.5 + scale_b)
-        out[f"quantize_{tag}"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
-                                  "algo_bytes": algo}
-        o_ = torch.empty(4096, 4096, dtype=torch.bfloat16, device=dev)
-        fn = lambda: q.qlora_nf4_dequantize(qw, o_)
-        for _ in range(3):
-            fn()
-        ms = graph_time(fn, 20, flush)
-        algo = ne * (0.5 + scale_b + 2.0)
-        out[f"dequantize_{tag}"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6,
-                                    "frac": algo / ms / 1e6 / peaks["hbm_gbs"], "algo_bytes": algo}
+    for qn, qk, sfx in ((4096, 4096, ""), (22016, 8192, "_65b_gate")):
+        _quant_components(q, synth, torch, dev, flush, peaks, out, qn, qk, sfx)
     # weight-stream bound forward at M = 16 (65B q_proj)
     n, k = 8192, 8192
     W = synth.weight(n, k).to(dev)

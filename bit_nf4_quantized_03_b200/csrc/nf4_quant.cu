@@ -75,8 +75,8 @@ __device__ __forceinline__ float absmax8(const float4& a, const float4& b) {
 }
 
 // Fixed pairwise tree (fp64) over part[0..n) zero-padded to a power of two,
-// by one CTA of 256 threads, without writing global memory (so every CTA of a
-// grid can run it on the same input). Each warp reduces an aligned group of
+// by one CTA (any multiple of 32 threads: the warps only share out the groups,
+// the tree is the same), without writing global memory. Each warp reduces an aligned group of
 // 512: every lane sums its 16 consecutive values pairwise, then five
 // xor-shuffle levels combine neighbouring lanes (a + b == b + a exactly, so
 // this is the same tree). The group sums go to shared memory and the next
@@ -93,7 +93,7 @@ __device__ double tree_sum_cta(const double* __restrict__ part, int64_t n, doubl
   while (n > 1) {
     const int64_t groups = (n + 511) / 512;
     double* dst = buf + pp * kTreeBuf;
-    for (int64_t g = warp; g < groups; g += 8) {
+    for (int64_t g = warp; g < groups; g += (blockDim.x >> 5)) {
       double v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -252,31 +252,35 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
 }
 
 // ---------------------------------------------------------------------------
-// Stage 2: the mean, then per 256-block d = a - mean, s2 = max|d| / 448,
-// q = e4m3(d / s2). Every CTA sums the per-chunk partials with the same fixed
-// tree (bit-identical results, no extra launch for the mean). Its up to
-// kFinishPer 256-blocks (one absmax per thread each) are requested before the
-// tree so the loads overlap it, and all of them are reduced in one barrier.
+// Stage 2: the mean, by one CTA of 1024 threads over the per-chunk partials
+// (the rest of the fixed tree), written to dq_mean.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) dq_mean_kernel(const double* __restrict__ part, int64_t nchunks,
+                                                       int64_t nblk, float* __restrict__ mean_out) {
+  __shared__ double tree_buf[2 * kTreeBuf];
+  const double S = tree_sum_cta(part, nchunks, tree_buf);
+  if (threadIdx.x == 0) *mean_out = static_cast<float>(S / static_cast<double>(nblk));
+}
+
+// ---------------------------------------------------------------------------
+// Stage 3: per 256-block d = a - mean, s2 = max|d| / 448, q = e4m3(d / s2).
+// Each CTA takes up to kFinishPer 256-blocks (one absmax per thread each),
+// requested together, and reduces all of them in one barrier.
 // ---------------------------------------------------------------------------
 constexpr int kFinishPer = 8;                 // 256-blocks per CTA, loaded up front
 
-__global__ void __launch_bounds__(256) dq_finish_kernel(const double* __restrict__ part, int64_t nchunks,
+__global__ void __launch_bounds__(256) dq_finish_kernel(const float* __restrict__ mean_in,
                                                          const float* __restrict__ absmax, int64_t nblk,
-                                                         uint8_t* __restrict__ q_out, float* __restrict__ s2_out,
-                                                         float* __restrict__ mean_out) {
-  __shared__ double tree_buf[2 * kTreeBuf];
+                                                         uint8_t* __restrict__ q_out, float* __restrict__ s2_out) {
   __shared__ float wmax[kFinishPer][8];
   const int64_t nb2 = (nblk + 255) / 256;
-  // this CTA's absmax values, requested before the mean so the loads overlap the tree
   float a[kFinishPer];
 #pragma unroll
   for (int j = 0; j < kFinishPer; ++j) {
     const int64_t b = (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(j) * gridDim.x) * 256 + threadIdx.x;
     a[j] = (b < nblk) ? __ldcg(absmax + b) : 0.f;
   }
-  const double S = tree_sum_cta(part, nchunks, tree_buf);
-  const float mean = static_cast<float>(S / static_cast<double>(nblk));
-  if (blockIdx.x == 0 && threadIdx.x == 0) *mean_out = mean;
+  const float mean = __ldcg(mean_in);
   float d[kFinishPer];
 #pragma unroll
   for (int j = 0; j < kFinishPer; ++j) {
@@ -460,13 +464,17 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // the rest of the tree, the mean and the E4M3 pass in one launch
+  // the rest of the tree and the mean (one CTA), then the E4M3 pass
+  dq_mean_kernel<<<1, 1024, 0, st>>>(part_a, nchunks, nblk, dq_mean);
+  count_launches(1);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const int64_t nb2 = (nblk + 255) / 256;
   // enough CTAs that each takes at most kFinishPer 256-blocks, at least one per SM when there is work
   int64_t g2 = (nb2 + kFinishPer - 1) / kFinishPer;
   if (g2 < num_sms) g2 = nb2 < num_sms ? nb2 : num_sms;
   const int grid2 = static_cast<int>(g2);
-  dq_finish_kernel<<<grid2, 256, 0, st>>>(part_a, nchunks, absmax, nblk, scale_fp8, dq_scale, dq_mean);
+  dq_finish_kernel<<<grid2, 256, 0, st>>>(dq_mean, absmax, nblk, scale_fp8, dq_scale);
   count_launches(1);
   return cudaGetLastError();
 }
