@@ -9,6 +9,8 @@
 // "Double quantization (the label-index-card trick)" stores the scales
 // themselves as 8-bit floats (E4M3) in blocks of 256 with one fp32 scale per
 // block and one fp32 mean offset per tensor.
+#include <cstring>
+
 #include "qlora_device.cuh"
 #include "qlora_kernels.h"
 
@@ -19,11 +21,14 @@ __device__ int g_device_error = 0;
 // ---------------------------------------------------------------------------
 // Stage 1: absmax, codes, plain scales / fp32 absmax for double quant.
 //
-// The weights stream through a 3-stage shared-memory ring filled by bulk
-// copies (32 KB chunks of 128 blocks). Eight lanes share one 64-block (eight
-// weights each, two conflict-free 128-bit shared reads), so the per-block
-// work -- absmax over the eight lanes, the IEEE reciprocal, the scale store --
-// is spread over eight weights per lane.
+// The weights stream through a 3-stage shared-memory ring filled by TMA: the
+// tensor is viewed as rows of one 64-block (256 B), and each 32 KB chunk of
+// 128 blocks arrives as two 128-row boxes of half-blocks, 128-byte swizzled,
+// so lanes reading the same offset of different blocks hit different banks.
+// Two lanes share one 64-block (32 weights each): one shuffle gives the
+// block's absmax, each lane takes the IEEE reciprocal and searches the codes
+// of its 32 weights (32 independent chains), and writes them as one 16-byte
+// store. A ragged last block is read from global memory.
 //
 // The code of x = w * (1/absmax) is found with one comparison: [-1 - 1/16,
 // 1 + 1/16) is cut into 35 buckets of width 1/16, each widened by 1e-3; the
@@ -35,11 +40,13 @@ __device__ int g_device_error = 0;
 //
 // In double-quant mode each chunk's 128 absmax values are also reduced in
 // fp64 with the fixed pairwise tree (the first levels of the tensor-wide sum
-// that defines the mean).
+// that defines the mean): 16 blocks per warp by shuffles, then the chunk's 8
+// warp sums.
 // ---------------------------------------------------------------------------
 constexpr int kQChunk = 128;     // 64-blocks per chunk: 32 KB of fp32 weights
 constexpr int kQStages = 3;
-constexpr int kQSmem = kQStages * kQChunk * 256;
+constexpr int kQStage = kQChunk * 256;                // bytes per stage: two 16 KB boxes of half-blocks
+constexpr int kQSmem = kQStages * kQStage + 1024;     // + alignment of the swizzled stages
 
 __device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2* tab) {
   // bucket = floor(x * 16 + 17): round-to-integer of x * 16 + 16.5 by adding 1.5 * 2^23
@@ -121,18 +128,25 @@ __device__ double tree_sum_cta(const double* __restrict__ part, int64_t n, doubl
 }
 
 template <bool kDQ>
-__global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __restrict__ W, int64_t n_elem,
+__global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                              const float* __restrict__ W, int64_t n_elem,
                                                               Nf4Buckets bk, uint8_t* __restrict__ codes,
                                                               uint16_t* __restrict__ scale_bf16,
                                                               float* __restrict__ absmax_out,
                                                               double* __restrict__ part_out) {
-  extern __shared__ __align__(128) uint8_t q_stage[];
+  extern __shared__ __align__(16) uint8_t q_raw[];    // aligned to 1024 below, at run time (the runtime places it after the static arrays)
+  uint8_t* q_stage = q_raw + ((1024u - (smem_u32(q_raw) & 1023u)) & 1023u);
+  if ((smem_u32(q_stage) & 1023u) != 0u) {   // the swizzled TMA boxes need a 1024-byte aligned stage
+    if (threadIdx.x == 0) atomicExch(&g_device_error, kErrBadLayout);
+    return;
+  }
   __shared__ float2 s_tab[64];
-  __shared__ double s_part[2][kQChunk / 4];   // per chunk: sums of 4 adjacent blocks (double-buffered by chunk)
+  __shared__ double s_part[2][8];             // per chunk: the eight warps' sums of 16 blocks (by chunk parity)
   __shared__ __align__(8) uint64_t full[kQStages];
   const int tid = threadIdx.x;
-  const int grp = tid >> 3;          // one 64-block per group of eight lanes
-  const int l = tid & 7;
+  const int h = tid & 1;                      // half of the block: elements 32h .. 32h + 31
+  const int lb = tid >> 1;                    // block within the chunk
+  const int warp = tid >> 5, lane = tid & 31;
   const int64_t nfull = n_elem / 64;
   const int64_t tail = n_elem - nfull * 64;
   const int64_t nblk = nfull + (tail > 0 ? 1 : 0);
@@ -147,104 +161,99 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const float* __res
   if (tid == 0) {
     for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
     fence_mbar_init();
+    if (nfull > 0) tma_prefetch_desc(&wmap);
   }
   __syncthreads();
   auto issue = [&](int64_t i) {
     const int64_t b0 = (blockIdx.x + i * gridDim.x) * kQChunk;
-    int64_t nb = nfull - b0;
-    nb = nb < 0 ? 0 : (nb > kQChunk ? kQChunk : nb);
     const int st = static_cast<int>(i % kQStages);
-    if (nb > 0) {
-      mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nb * 256));
-      bulk_load(q_stage + st * (kQChunk * 256), W + b0 * 64, static_cast<uint32_t>(nb * 256), &full[st]);
+    if (b0 < nfull) {
+      // rows past nfull arrive zero-filled and are counted in full
+      uint8_t* dst = q_stage + st * kQStage;
+      mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(kQStage));
+      tma_load_2d(dst, &wmap, &full[st], 0, static_cast<int32_t>(b0));
+      tma_load_2d(dst + kQStage / 2, &wmap, &full[st], 32, static_cast<int32_t>(b0));
     } else {
-      mbar_arrive(&full[st]);
+      mbar_arrive(&full[st]);                  // only the ragged last block: read from global memory
     }
   };
   if (tid == 0)
     for (int64_t i = 0; i < my_n && i < kQStages; ++i) issue(i);
-  // Lanes 4..7 of a group read the second half of their 32 bytes first, so the
-  // eight lanes of a quarter-warp hit eight different bank groups.
-  const uint32_t x = (l >> 2) & 1;
-  const uint32_t sh_first = 16 * x, sh_second = 16 * (x ^ 1);
+  const uint32_t swz = static_cast<uint32_t>(lb & 7);       // 128-byte swizzle of this lane's row
   for (int64_t i = 0; i < my_n; ++i) {
     const int st = static_cast<int>(i % kQStages);
     if (!mbar_wait(&full[st], static_cast<uint32_t>((i / kQStages) & 1))) break;
     const int64_t b0 = (blockIdx.x + i * gridDim.x) * kQChunk;
-    const uint32_t sbase = smem_u32(q_stage + st * (kQChunk * 256)) + l * 32;
-    const bool whole = (b0 + kQChunk <= nfull);
-#pragma unroll 2
-    for (int it = 0; it < kQChunk / 32; ++it) {
-      const int lb = it * 32 + grp;
-      const int64_t b = b0 + lb;
-      uint32_t word;
-      float m;
-      if (whole || b < nfull) {
-        float4 f, g;   // f: elements of the half read first, g: the other half
-        const uint32_t src = sbase + lb * 256;
+    const int64_t b = b0 + lb;
+    // block class: 0 = whole block in the stage, 1 = ragged last block, 2 = past the tensor
+    const int cls = (b < nfull) ? 0 : ((b == nfull && tail > 0) ? 1 : 2);
+    float4 v[8];
+    if (cls == 0) {
+      const uint32_t row = smem_u32(q_stage + st * kQStage + h * (kQStage / 2)) + static_cast<uint32_t>(lb) * 128u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
         asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(src + sh_first) : "memory");
-        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(g.x), "=f"(g.y), "=f"(g.z), "=f"(g.w) : "r"(src + sh_second) : "memory");
-        m = absmax8(f, g);
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-        word = 0x77777777u;               // zero or subnormal absmax: the exact-zero level
-        if (m >= 1.17549435e-38f) {
-          const uint32_t w = nf4_codes8(f, g, __frcp_rn(m), s_tab);   // f -> nibbles 0..3, g -> 4..7
-          word = x ? ((w << 16) | (w >> 16)) : w;                    // back to element order
-        }
-        reinterpret_cast<uint32_t*>(codes)[b * 8 + l] = word;
-      } else {
-        float4 f, g;
-        float* fv = reinterpret_cast<float*>(&f);
-        float* gv = reinterpret_cast<float*>(&g);
+                     : "=f"(v[c].x), "=f"(v[c].y), "=f"(v[c].z), "=f"(v[c].w)
+                     : "r"(row + ((static_cast<uint32_t>(c) ^ swz) << 4))
+                     : "memory");
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float* f = reinterpret_cast<float*>(&v[c]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int64_t i0 = 8 * l + e, i1 = 8 * l + 4 + e;
-          fv[e] = (b == nfull && i0 < tail) ? W[b * 64 + i0] : 0.f;
-          gv[e] = (b == nfull && i1 < tail) ? W[b * 64 + i1] : 0.f;
+          const int64_t el = 32 * h + 4 * c + e;
+          f[e] = (cls == 1 && el < tail) ? W[b * 64 + el] : 0.f;
         }
-        m = absmax8(f, g);
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-        word = 0x77777777u;
-        if (m >= 1.17549435e-38f) word = nf4_codes8(f, g, __frcp_rn(m), s_tab);
-        if (b == nfull && tail > 0) {
-          // ragged last block: only the bytes that hold present elements; an odd tail keeps its high nibble 0
-#pragma unroll
-          for (int byte = 0; byte < 4; ++byte) {
-            const int64_t e0 = 8 * l + 2 * byte;
-            if (e0 < tail) {
-              uint32_t c = (word >> (8 * byte)) & 0xFFu;
-              if (e0 + 1 >= tail) c &= 0x0Fu;
-              codes[b * 32 + 4 * l + byte] = static_cast<uint8_t>(c);
-            }
-          }
-        }
-      }
-      if (l == 0 && b < nblk) {
-        if (kDQ) absmax_out[b] = m;
-        else scale_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
-      }
-      if (kDQ) {
-        // first two levels of the fixed pairwise tree: the warp's four groups hold four
-        // adjacent blocks (lb = it*32 + 4*warp + 0..3), all eight lanes of a group hold its m
-        double t = (b < nblk) ? static_cast<double>(m) : 0.0;
-        t = t + __shfl_xor_sync(0xffffffffu, t, 8);
-        t = t + __shfl_xor_sync(0xffffffffu, t, 16);
-        if ((tid & 31) == 0) s_part[i & 1][it * 8 + (tid >> 5)] = t;
       }
     }
-    fence_proxy_async_smem();                 // reads of the stage ordered before its bulk-copy refill
+    float m = fmaxf(fmaxf(absmax8(v[0], v[1]), absmax8(v[2], v[3])), fmaxf(absmax8(v[4], v[5]), absmax8(v[6], v[7])));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));     // the partner lane holds the other half
+    uint4 word = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);  // zero or subnormal absmax
+    if (cls != 2 && m >= 1.17549435e-38f) {
+      const float inv = __frcp_rn(m);
+      word.x = nf4_codes8(v[0], v[1], inv, s_tab);
+      word.y = nf4_codes8(v[2], v[3], inv, s_tab);
+      word.z = nf4_codes8(v[4], v[5], inv, s_tab);
+      word.w = nf4_codes8(v[6], v[7], inv, s_tab);
+    }
+    if (cls == 0) {
+      *reinterpret_cast<uint4*>(codes + b * 32 + h * 16) = word;
+    } else if (cls == 1) {
+      // only the bytes that hold present elements; an odd tail keeps its high nibble 0
+      const uint32_t ww[4] = {word.x, word.y, word.z, word.w};
+#pragma unroll
+      for (int byte = 0; byte < 16; ++byte) {
+        const int64_t e0 = 32 * h + 2 * byte;
+        if (e0 < tail) {
+          uint32_t c = (ww[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
+          if (e0 + 1 >= tail) c &= 0x0Fu;
+          codes[b * 32 + 16 * h + byte] = static_cast<uint8_t>(c);
+        }
+      }
+    }
+    if (h == 0 && b < nblk) {
+      if (kDQ) absmax_out[b] = m;
+      else scale_bf16[b] = __bfloat16_as_ushort(__float2bfloat16_rn(m));
+    }
+    if (kDQ) {
+      // first four levels of the fixed pairwise tree over the warp's 16 adjacent blocks
+      // (lane 2j + h holds block 16 * warp + j; both lanes of a block hold its absmax)
+      double t = (b < nblk) ? static_cast<double>(m) : 0.0;
+      t = t + __shfl_xor_sync(0xffffffffu, t, 2);
+      t = t + __shfl_xor_sync(0xffffffffu, t, 4);
+      t = t + __shfl_xor_sync(0xffffffffu, t, 8);
+      t = t + __shfl_xor_sync(0xffffffffu, t, 16);
+      if (lane == 0) s_part[i & 1][warp] = t;
+    }
+    fence_proxy_async_smem();                 // reads of the stage ordered before its refill
     __syncthreads();                          // stage consumed, tree nodes written
     if (kDQ && tid < 32) {
-      // remaining five levels over the chunk's 32 nodes, in index order (xor-shuffle pairs)
-      double t = s_part[i & 1][tid];
+      // remaining three levels over the chunk's 8 warp sums, in index order (xor-shuffle pairs)
+      double t = (tid < 8) ? s_part[i & 1][tid] : 0.0;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
+      for (int off = 1; off < 8; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
       if (tid == 0) part_out[blockIdx.x + i * gridDim.x] = t;
     }
     if (tid == 0 && i + kQStages < my_n) issue(i + kQStages);
@@ -446,11 +455,18 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   const bool dq = (scale_fp8 != nullptr);
   const int64_t nchunks = (nblk + kQChunk - 1) / kQChunk;
   const int grid = static_cast<int>(nchunks < 2LL * num_sms ? nchunks : 2LL * num_sms);
+  // W as rows of one 64-block; boxes of 128 rows x 32 floats (128 B, swizzled)
+  CUtensorMap wmap;
+  std::memset(&wmap, 0, sizeof(wmap));
+  const int64_t nfull = n_elem / 64;
+  if (nfull > 0 && !tmap_2d(&wmap, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 64, static_cast<uint64_t>(nfull), 256, 32,
+                            kQChunk, 128))
+    return cudaErrorInvalidValue;
   cudaError_t e;
   if (!dq) {
     e = set_smem_once(nf4_quantize_kernel<false>, kQSmem, smem_set[0]);
     if (e != cudaSuccess) return e;
-    nf4_quantize_kernel<false><<<grid, 256, kQSmem, st>>>(W, n_elem, bk, codes, scale_bf16, nullptr, nullptr);
+    nf4_quantize_kernel<false><<<grid, 256, kQSmem, st>>>(wmap, W, n_elem, bk, codes, scale_bf16, nullptr, nullptr);
     count_launches(1);
     return cudaGetLastError();
   }
@@ -460,7 +476,7 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   // stage 1 also writes one fp64 tree sum per chunk (the first levels of the fixed-order sum)
   e = set_smem_once(nf4_quantize_kernel<true>, kQSmem, smem_set[1]);
   if (e != cudaSuccess) return e;
-  nf4_quantize_kernel<true><<<grid, 256, kQSmem, st>>>(W, n_elem, bk, codes, nullptr, absmax, part_a);
+  nf4_quantize_kernel<true><<<grid, 256, kQSmem, st>>>(wmap, W, n_elem, bk, codes, nullptr, absmax, part_a);
   count_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

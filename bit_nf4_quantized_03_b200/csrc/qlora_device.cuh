@@ -31,7 +31,7 @@ struct Nf4Buckets {
 
 // Device error word: kernels write a non-zero code here when a bounded wait
 // gives up, so the host can read the failure instead of the GPU hanging.
-enum : int { kErrNone = 0, kErrWaitTimeout = 1 };
+enum : int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadLayout = 2 };   // values of g_device_error
 extern __device__ int g_device_error;
 
 // ---------------------------------------------------------------------------
