@@ -83,10 +83,12 @@ __device__ __forceinline__ float absmax8(const float4& a, const float4& b) {
 
 // Fixed pairwise tree (fp64) over part[0..n) zero-padded to a power of two,
 // by one CTA (any multiple of 32 threads: the warps only share out the groups,
-// the tree is the same), without writing global memory. Each warp reduces an aligned group of
-// 512: every lane sums its 16 consecutive values pairwise, then five
-// xor-shuffle levels combine neighbouring lanes (a + b == b + a exactly, so
-// this is the same tree). The group sums go to shared memory and the next
+// the tree is the same), without writing global memory. Each warp reduces an
+// aligned group of 512: lane l loads elements l, l + 32, ..., l + 480 of the
+// group (coalesced); five xor-shuffle levels sum each aligned run of 32
+// (neighbouring elements sit in neighbouring lanes, and a + b == b + a
+// exactly, so each node is the same left + right), and four levels inside the
+// lane pair up the 16 runs. The group sums go to shared memory and the next
 // level runs on them, until one value is left. Zero padding at any level
 // leaves the result unchanged (x + 0 == x), so this equals the tree over the
 // whole power-of-two-padded array. `buf` holds 2 * kTreeBuf doubles.
@@ -104,17 +106,18 @@ __device__ double tree_sum_cta(const double* __restrict__ part, int64_t n, doubl
       double v[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int64_t idx = g * 512 + lane * 16 + j;
+        const int64_t idx = g * 512 + j * 32 + lane;
         v[j] = (idx < n) ? (global_src ? __ldcg(src + idx) : src[idx]) : 0.0;
       }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = v[j] + __shfl_xor_sync(0xffffffffu, v[j], off);
 #pragma unroll
       for (int w = 1; w < 16; w <<= 1)
 #pragma unroll
         for (int j = 0; j < 16; j += 2 * w) v[j] = v[j] + v[j + w];
-      double t = v[0];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
-      if (lane == 0) dst[g] = t;
+      if (lane == 0) dst[g] = v[0];
     }
     __syncthreads();
     src = dst;
@@ -249,6 +252,7 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const __grid_const
     }
     fence_proxy_async_smem();                 // reads of the stage ordered before its refill
     __syncthreads();                          // stage consumed, tree nodes written
+    if (tid == 0 && i + kQStages < my_n) issue(i + kQStages);
     if (kDQ && tid < 32) {
       // remaining three levels over the chunk's 8 warp sums, in index order (xor-shuffle pairs)
       double t = (tid < 8) ? s_part[i & 1][tid] : 0.0;
@@ -256,7 +260,6 @@ __global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const __grid_const
       for (int off = 1; off < 8; off <<= 1) t = t + __shfl_xor_sync(0xffffffffu, t, off);
       if (tid == 0) part_out[blockIdx.x + i * gridDim.x] = t;
     }
-    if (tid == 0 && i + kQStages < my_n) issue(i + kQStages);
   }
 }
 
