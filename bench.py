@@ -51,7 +51,7 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
 # recorded with it; any change to them prints null until the counters are taken again.
 WGEMM_TRAFFIC = {"bytes_per_launch": 910676891,
-                 "sources_sha256": "395e3aac4dca070a4dd98d35bd98389747527a92fc9972e376690d764b9899f9"}
+                 "sources_sha256": "06d35cbb1e37d19ce49c067e21bcb25cc5b2284cc6b1a9e91970093f1bcbbecf"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 
@@ -639,6 +639,12 @@ def run_case(args) -> None:
         wm = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
         for _ in range(1 + args.case_iters):
             q.qlora_lora_merge(qw, a, b, RANK_R, ALPHA, wm, q.QLORA_DTYPE_BF16)
+    elif name == "quantize_8192":
+        # plain (BF16-scale) quantize of a 65B q/k/v/o-shaped weight
+        W = synth.weight(8192, 8192, outlier_frac=0.001).to(dev)
+        qw = q.QuantizedWeight(8192, 8192, q.QLORA_SCALE_BF16, device=dev)
+        for _ in range(1 + args.case_iters):
+            q.qlora_nf4_quantize(W, qw)
     elif name in ("quantize_4096", "dequantize_4096"):
         W = synth.weight(4096, 4096, outlier_frac=0.001).to(dev)
         qw = q.QuantizedWeight(4096, 4096, q.QLORA_SCALE_DQ_FP8, device=dev)
