@@ -557,7 +557,12 @@ struct PCfg {
   // Dequantizer groups of four warps: group g expands the main K steps whose ring
   // index is g modulo kGroups, so kGroups steps are in expansion at once.
   static constexpr int Groups = kGroups;
-  static constexpr int kThreads = (6 + 4 * kGroups) * 32;
+  // Epilogue warps: four (one per TMEM lane quarter) draining every column, or eight,
+  // two per quarter each draining half the columns (the second four after the dequantizers).
+  static constexpr int EpiWarps = (kNT == 2) ? 8 : 4;
+  static constexpr int kDeqWarp0 = 6;
+  static constexpr int kEpi2Warp0 = 6 + 4 * kGroups;
+  static constexpr int kThreads = (6 + 4 * kGroups + (EpiWarps - 4)) * 32;
   static constexpr int kTmemCols = 512;      // two accumulators of 256 columns
   static constexpr int kBStage = NT * kBTile;  // activation bytes of one stage in one CTA
   static constexpr int kSmemBytes = Stages * (kATile + kBStage + kRBytes) + 1024 + 256;
@@ -603,7 +608,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 8);
+      mbar_init(&acc_empty[a], 2 * C::EpiWarps);    // every epilogue warp of both CTAs
     }
     fence_mbar_init();
   }
@@ -729,9 +734,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < C::kDeqWarp0 || warp >= C::kEpi2Warp0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
+    const int q = warp & 3;                                           // TMEM lane quarter
+    constexpr int kCols = C::TOK / (C::EpiWarps / 4);                 // columns per warp
+    const int col0 = (warp >= C::kEpi2Warp0) ? kCols : 0;
     const uint32_t acc_empty_e0 = smem_cluster_addr(&acc_empty[0], 0);
     const uint32_t acc_empty_e1 = smem_cluster_addr(&acc_empty[1], 0);
     int acc = 0;
@@ -744,11 +751,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       const int feat = (2 * mb + rank) * 128 + q * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::TOK);
 #pragma unroll 1
-      for (int c = 0; c < C::TOK / 32; ++c) {
+      for (int c = col0; c < col0 + kCols; c += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
+        tmem_ld_32x32b_x32(t_row + c, v);
         tmem_ld_wait();
-        wstore<32>(p, split, feat, nb * C::TOK + c * 32, v);
+        wstore<32>(p, split, feat, nb * C::TOK + c, v);
       }
       tc_fence_before();
       __syncwarp();
@@ -759,8 +766,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // ------------------------------------------------------------ dequantizers (both CTAs)
     // As in the single-CTA kernel, on this CTA's 128-row tile, with C::Groups groups taking
     // main K steps in turn; each warp reports its finished tile to the even CTA's deq_full.
-    const int grp = (warp - 6) >> 2;
-    const int gt = threadIdx.x - 192 - 128 * grp;    // 0..127
+    const int grp = (warp - C::kDeqWarp0) >> 2;
+    const int gt = threadIdx.x - 32 * C::kDeqWarp0 - 128 * grp;    // 0..127
     const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
     const int i_mn = gt & 63;
     const int c_mn = gt >> 6;
