@@ -50,8 +50,8 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum; summary in
 # profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
 # recorded with it; any change to them prints null until the counters are taken again.
-WGEMM_TRAFFIC = {"bytes_per_launch": 910676891,
-                 "sources_sha256": "6dec3f93b5c15a21052d2882a74dec6096d87d893222b43b9835fe14c206bedc"}
+WGEMM_TRAFFIC = {"bytes_per_launch": 924497618,
+                 "sources_sha256": "bc0c998b989d9181068014875f03cf209df3f4c854e6691ec19df981fd754522"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 
