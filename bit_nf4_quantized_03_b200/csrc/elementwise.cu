@@ -106,35 +106,56 @@ cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_str
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
                                      int64_t cols, int64_t ld_part, void* __restrict__ out, int out_bf16,
                                      int accumulate) {
-  const int64_t c4 = cols / 4;
-  const int64_t total = rows * c4;
+  // eight consecutive columns per thread (cols % 8 == 0): two 16-byte partial loads per
+  // split and one 16-byte BF16 (or two fp32) accesses of the output
+  const int64_t c8 = cols / 8;
+  const int64_t total = rows * c8;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = idx / c4;
-    const int64_t col = (idx - row * c4) * 4;
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t row = idx / c8;
+    const int64_t col = (idx - row * c8) * 8;
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int t = 0; t < splits; ++t) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(part + t * part_stride + row * ld_part + col));
-      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      const float4* src = reinterpret_cast<const float4*>(part + t * part_stride + row * ld_part + col);
+      const float4 a = __ldcs(src);
+      const float4 b = __ldcs(src + 1);
+      s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
+      s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
     }
     if (out_bf16) {
-      uint16_t* o = static_cast<uint16_t*>(out) + row * cols + col;
-      if (accumulate) { s.x += bf2f(o[0]); s.y += bf2f(o[1]); s.z += bf2f(o[2]); s.w += bf2f(o[3]); }
-      uint2 w;
-      w.x = pack_bf16x2(s.x, s.y);
-      w.y = pack_bf16x2(s.z, s.w);
-      *reinterpret_cast<uint2*>(o) = w;
+      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row * cols + col);
+      if (accumulate) {
+        const uint4 y = *o;
+        const uint32_t w[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          s[2 * j] += __uint_as_float(w[j] << 16);
+          s[2 * j + 1] += __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      }
+      uint4 r;
+      r.x = pack_bf16x2(s[0], s[1]);
+      r.y = pack_bf16x2(s[2], s[3]);
+      r.z = pack_bf16x2(s[4], s[5]);
+      r.w = pack_bf16x2(s[6], s[7]);
+      *o = r;
     } else {
       float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + row * cols + col);
-      if (accumulate) { const float4 y = *o; s.x += y.x; s.y += y.y; s.z += y.z; s.w += y.w; }
-      *o = s;
+      if (accumulate) {
+        const float4 y0 = o[0], y1 = o[1];
+        s[0] += y0.x; s[1] += y0.y; s[2] += y0.z; s[3] += y0.w;
+        s[4] += y1.x; s[5] += y1.y; s[6] += y1.z; s[7] += y1.w;
+      }
+      o[0] = make_float4(s[0], s[1], s[2], s[3]);
+      o[1] = make_float4(s[4], s[5], s[6], s[7]);
     }
   }
 }
 
 cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_stride, int64_t rows, int64_t cols,
                                  int64_t ld_part, void* out, int out_bf16, int accumulate, cudaStream_t st) {
-  splitk_reduce_kernel<<<blocks_for(rows * (cols / 4), 256), 256, 0, st>>>(part, splits, part_stride, rows, cols,
+  if (cols % 8 != 0 || ld_part % 8 != 0) return cudaErrorInvalidValue;
+  splitk_reduce_kernel<<<blocks_for(rows * (cols / 8), 256), 256, 0, st>>>(part, splits, part_stride, rows, cols,
                                                                             ld_part, out, out_bf16, accumulate);
   count_launches(1);
   return cudaGetLastError();
