@@ -252,15 +252,17 @@ class Workload:
             self.w[name], self.A[name], self.B[name] = qw, a.to(dev), b.to(dev)
         torch.cuda.synchronize()
         M, H, I = M_TOKENS, 8192, 22016
-        # host copies (pinned) of every input a step consumes
+        # host copies (pinned) of every input a step consumes, in the order the step first reads them
         self.host = {
             "x_attn": synth.activations(M, H, layer=off + 10), "x_o": synth.activations(M, H, layer=off + 11),
-            "x_mlp": synth.activations(M, H, layer=off + 12),
-            "dy_q": synth.grad_output(M, H, layer=off + 20), "dy_k": synth.grad_output(M, H, layer=off + 21),
-            "dy_v": synth.grad_output(M, H, layer=off + 22), "dy_o": synth.grad_output(M, H, layer=off + 23),
-            "dy_mlp": synth.grad_output(M, H, layer=off + 24),
+            "x_mlp": synth.activations(M, H, layer=off + 12), "dy_mlp": synth.grad_output(M, H, layer=off + 24),
+            "dy_o": synth.grad_output(M, H, layer=off + 23), "dy_q": synth.grad_output(M, H, layer=off + 20),
+            "dy_k": synth.grad_output(M, H, layer=off + 21), "dy_v": synth.grad_output(M, H, layer=off + 22),
             "x16": synth.activations(M_SMALL, H, layer=off + 30), "h16": synth.activations(M_SMALL, I, layer=off + 31),
         }
+        # per-input copy events of the current input set (end-to-end timing only): the step
+        # waits for each input just before its first use
+        self.in_events = None
         self.host = {k_: v.pin_memory() for k_, v in self.host.items()}
         self.d = {k_: v.to(dev) for k_, v in self.host.items()}
         e = lambda *s, dt=bf: torch.empty(*s, dtype=dt, device=dev)
@@ -296,8 +298,21 @@ class Workload:
         q.qlora_linear_bwd(self.w[nm], X, dY, self.A[nm], self.B[nm], RANK_R, ALPHA, self.U[nm], dX,
                            q.QLORA_DTYPE_BF16, self.dA[nm], self.dB[nm], flags, self.ws)
 
+    def _inputs(self):
+        """The input set, as a mapping whose lookup first makes the compute stream wait
+        for that input's host copy when one is in flight."""
+        import torch
+        d, evs = self.d, self.in_events
+
+        class _Waiting:
+            def __getitem__(self, key):
+                if evs is not None:
+                    torch.cuda.current_stream().wait_event(evs[key])
+                return d[key]
+        return d if evs is None else _Waiting()
+
     def step(self):
-        q, d = self.q, self.d
+        q, d = self.q, self._inputs()
         for nm in ("q_proj", "k_proj", "v_proj"):
             self._fwd(nm, d["x_attn"], self.y[nm], self.U[nm])
         self._fwd("o_proj", d["x_o"], self.y["o_proj"], self.U["o_proj"])
@@ -331,15 +346,25 @@ def time_e2e_pipelined(wl, steps, sync_barrier=None):
     the pinned-host inputs of step i+1 go to a second device input set on a copy stream
     while step i computes, and step i's adapter gradients are copied device-side to a
     staging buffer (so step i+1 cannot overwrite them) and read back to pinned host
-    memory on the copy stream. Timed by CUDA events from the first copy to the last
-    read-back; the inputs of every step exceed L2, so nothing is flushed in between."""
+    memory on a third stream, so the read-back never queues behind the next input
+    copy (the two directions use separate copy engines). Timed by CUDA events from
+    the first copy to the last read-back; the inputs of every step exceed L2, so
+    nothing is flushed in between."""
     import torch
     comp = torch.cuda.current_stream()
     cs = torch.cuda.Stream()
+    rs = torch.cuda.Stream()
     sets = [wl.d, {k_: torch.empty_like(v) for k_, v in wl.d.items()}]
     stage = [torch.empty_like(wl.grads), torch.empty_like(wl.grads)]
     ev = lambda: torch.cuda.Event()
-    copied, done, staged, read = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    done, staged, read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    copied = [{k_: ev() for k_ in wl.host}, {k_: ev() for k_ in wl.host}]   # one event per input and set
+
+    def copy_inputs(dst):
+        for k_, v in wl.host.items():
+            sets[dst][k_].copy_(v, non_blocking=True)
+            copied[dst][k_].record(cs)
+
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     base = wl.d
     if sync_barrier:
@@ -348,37 +373,52 @@ def time_e2e_pipelined(wl, steps, sync_barrier=None):
     t0.record(comp)
     cs.wait_event(t0)
     with torch.cuda.stream(cs):
-        for k_, v in wl.host.items():
-            sets[0][k_].copy_(v, non_blocking=True)
-        copied[0].record(cs)
+        copy_inputs(0)
     for i in range(steps):
         cur, nxt = i % 2, (i + 1) % 2
         if i + 1 < steps:
             with torch.cuda.stream(cs):
                 if i >= 1:
                     cs.wait_event(done[nxt])          # step i-1 is finished with that input set
-                for k_, v in wl.host.items():
-                    sets[nxt][k_].copy_(v, non_blocking=True)
-                copied[nxt].record(cs)
-        comp.wait_event(copied[cur])
+                copy_inputs(nxt)
         if i >= 2:
             comp.wait_event(read[cur])                # staging buffer free again
-        wl.d = sets[cur]
+        wl.d, wl.in_events = sets[cur], copied[cur]   # the step waits on each input before its first use
         wl.step()
+        wl.in_events = None
         done[cur].record(comp)
         stage[cur].copy_(wl.grads, non_blocking=True)
         staged[cur].record(comp)
-        with torch.cuda.stream(cs):
-            cs.wait_event(staged[cur])
+        with torch.cuda.stream(rs):
+            rs.wait_event(staged[cur])
             wl.host_grads.copy_(stage[cur], non_blocking=True)
-            read[cur].record(cs)
+            read[cur].record(rs)
     comp.wait_stream(cs)
+    comp.wait_stream(rs)
     t1.record(comp)
     torch.cuda.synchronize()
     wl.d = base
     if sync_barrier:
         sync_barrier()
     return t0.elapsed_time(t1) / steps
+
+
+def time_h2d_alone(wl, reps, sync_barrier=None):
+    """Device time of one step's pinned-host input copies with no compute beside them
+    (the floor of the end-to-end step when the host link is the bottleneck)."""
+    import torch
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sync_barrier:
+        sync_barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(reps):
+        wl.h2d()
+    t1.record()
+    torch.cuda.synchronize()
+    if sync_barrier:
+        sync_barrier()
+    return t0.elapsed_time(t1) / reps
 
 
 def time_steps(fn, steps, flush=None, sync_barrier=None):
@@ -718,10 +758,14 @@ def run_native(args) -> None:
         for _ in range(2):
             e2e_step()
         ms_e2e = max_over_ranks(time_e2e_pipelined(wl, args.steps, barrier))
+        ms_h2d = max_over_ranks(time_h2d_alone(wl, 3, barrier))
         e2e = {"value": flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": wl.h2d_bytes,
                "d2h_bytes_per_step": wl.d2h_bytes, "ms_per_step": ms_e2e,
-               "copies": "every step's inputs H2D from pinned host and its adapter gradients D2H, on a copy "
-                         "stream overlapped with the neighbouring step's compute (double-buffered)"}
+               "h2d_alone_ms": ms_h2d, "h2d_alone_gbs": wl.h2d_bytes / (ms_h2d * 1e-3) / 1e9,
+               "copies": "every step's inputs H2D from pinned host on a copy stream and its adapter gradients D2H "
+                         "on a second one, both overlapped with the neighbouring step's compute (double-buffered); "
+                         "each input is awaited just before its first use, so the first step starts once its first "
+                         "input has landed; h2d_alone_ms is one step's input copies with nothing else running"}
 
     peak_tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None

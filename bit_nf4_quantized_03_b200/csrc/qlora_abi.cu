@@ -168,14 +168,32 @@ struct Split {
   int splits = 1, kps = 1;
 };
 
-Split choose_split(int64_t tiles, int64_t k_tiles, int sms) {
-  Split s;
-  int64_t want = std::max<int64_t>(1, sms / std::max<int64_t>(tiles, 1));
-  want = std::min<int64_t>(want, std::max<int64_t>(k_tiles, 1));
-  want = std::min<int64_t>(want, 64);
-  s.kps = static_cast<int>(cdiv(std::max<int64_t>(k_tiles, 1), want));
-  s.splits = static_cast<int>(cdiv(std::max<int64_t>(k_tiles, 1), s.kps));
-  return s;
+// Split of a low-rank GEMM's reduction (U, G, dB, dA) over a persistent grid of
+// `sms` CTAs. These stream one 128 x 64 bf16 tile of the large operand per K step,
+// so the makespan in K steps is the number of waves times the steps per unit; each
+// split adds one fp32 partial of the [out_elems] result, written once and read
+// once, mostly from L2 (charged at half the weight of HBM traffic). Few tiles over
+// many SMs need a split to fill the grid; tiles just above the SM count need one
+// to even out the last wave.
+Split choose_lsplit(int64_t tiles, int64_t k_tiles, int sms, int64_t out_elems) {
+  const double bytes_per_wave_step = static_cast<double>(sms) * 16384.0;
+  Split best;
+  best.kps = static_cast<int>(std::max<int64_t>(k_tiles, 1));
+  best.splits = 1;
+  double best_cost = 1e300;
+  for (int64_t want = 1; want <= std::min<int64_t>(64, std::max<int64_t>(k_tiles, 1)); ++want) {
+    const int64_t kps = cdiv(std::max<int64_t>(k_tiles, 1), want);
+    const int64_t splits = cdiv(std::max<int64_t>(k_tiles, 1), kps);
+    const int64_t waves = cdiv(std::max<int64_t>(tiles, 1) * splits, sms);
+    double cost = static_cast<double>(waves) * (static_cast<double>(kps) + 1.0);
+    if (splits > 1) cost += static_cast<double>(splits) * static_cast<double>(out_elems) * 4.0 / bytes_per_wave_step;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best.kps = static_cast<int>(kps);
+      best.splits = static_cast<int>(splits);
+    }
+  }
+  return best;
 }
 
 // Split of the fused GEMM's reduction over a persistent grid of `sms` CTAs:
@@ -223,10 +241,11 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
     P.grad = kGemmLoraGrad128;
   }
   const int64_t tm = cdiv(m, 128);
-  P.u = choose_split(tm, k / 64, sms);
-  P.g = choose_split(tm, cdiv(n, 64), sms);
-  P.db = choose_split(cdiv(n, 128), cdiv(m, 64), sms);
-  P.da = choose_split(cdiv(k, 128), cdiv(m, 64), sms);
+  const int64_t rp64 = P.r_pad;
+  P.u = choose_lsplit(tm, k / 64, sms, m * rp64);
+  P.g = choose_lsplit(tm, cdiv(n, 64), sms, m * rp64);
+  P.db = choose_lsplit(cdiv(n, 128), cdiv(m, 64), sms, n * rp64);
+  P.da = choose_lsplit(cdiv(k, 128), cdiv(m, 64), sms, k * rp64);
   P.bn = wgemm_bn(m);
   const int64_t tok_tiles = cdiv(m, P.bn);
   const int64_t wrows = wgemm_tile_rows(P.bn);
