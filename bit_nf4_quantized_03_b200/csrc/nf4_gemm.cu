@@ -22,7 +22,7 @@
 
 namespace qlora {
 
-template <int kBN, int kStages, bool kAMn, int kBMode, bool kExt, bool kHiLo>
+template <int kBN, int kStages, bool kAMn, int kBMode, bool kExt, bool kHiLo, int kEpiGroups = 1>
 struct GemmCfg {
   static constexpr int BN = kBN;
   static constexpr int Stages = kStages;
@@ -34,12 +34,17 @@ struct GemmCfg {
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBTile = BN * 64 * 2;
   static constexpr int kBBytes = kBTile * (HiLo ? 2 : 1);
-  static constexpr int kThreads = 6 * 32;
+  // Epilogue warp groups: 1 = warps 2-5 drain both accumulator buffers in turn; 2 = warps
+  // 2-5 drain buffer 0 and warps 6-9 buffer 1, so two units' output round trips overlap
+  // (the masked dX pass, whose units are one K step each and bound by that round trip).
+  static constexpr int EpiGroups = kEpiGroups;
+  static constexpr int kThreads = (2 + 4 * kEpiGroups) * 32;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kBarBytes = 256;
-  static constexpr int kEpiStage = 4 * 32 * 32 * 4;   // one 32 x 32 fp32 chunk per epilogue warp (masked modes)
+  static constexpr int kEpiStage = 4 * kEpiGroups * 32 * 32 * 4;   // one 32 x 32 fp32 chunk per epilogue warp
   static constexpr int kSmemBytes = Stages * (kABytes + kBBytes) + kEpiStage + 1024 + kBarBytes;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM alloc size");
+  static_assert(kEpiGroups == 1 || kEpiGroups == 2, "one epilogue group per accumulator buffer at most");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -143,20 +148,20 @@ __device__ __forceinline__ void store_row32(const GemmParams& p, int split, int 
 // and mask byte of the unit is requested first (one memory round trip per unit); then
 // each 32-column chunk of the accumulator goes through a 128B-swizzled fp32 staging tile
 // so that four lanes share one output row and every access covers 8 rows x 64 bytes.
-template <int NCH>
+template <int NCH, bool f32>
 __device__ __forceinline__ void masked_acc_unit(const GemmParams& p, uint32_t stage, int lane, int row0, int col0,
                                                 uint32_t t_row) {
   const int sub = lane >> 2;            // row within a pass of 8 rows
   const int cc = (lane & 3) * 8;        // first of this lane's eight columns within a chunk
-  const bool f32 = (p.out_mode == kOutMaskAccF32);
-  uint4 y[NCH][4], y2[NCH][4];
+  uint4 y[NCH][4], y2[f32 ? NCH : 1][4];
   uint32_t bits[NCH][4];
 #pragma unroll
   for (int c = 0; c < NCH; ++c)
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int row = row0 + pass * 8 + sub;
-      y[c][pass] = y2[c][pass] = make_uint4(0u, 0u, 0u, 0u);
+      y[c][pass] = make_uint4(0u, 0u, 0u, 0u);
+      if (f32) y2[f32 ? c : 0][pass] = make_uint4(0u, 0u, 0u, 0u);
       bits[c][pass] = 0u;
       // a group of eight columns lies wholly inside or wholly outside the row (cols % 64 == 0)
       if (row < p.rows && col0 + c * 32 + cc < p.cols) {
@@ -165,7 +170,7 @@ __device__ __forceinline__ void masked_acc_unit(const GemmParams& p, uint32_t st
         if (f32) {
           const uint4* o = reinterpret_cast<const uint4*>(static_cast<const float*>(p.out) + e0);
           y[c][pass] = o[0];
-          y2[c][pass] = o[1];
+          y2[f32 ? c : 0][pass] = o[1];
         } else {
           y[c][pass] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.out) + e0);
         }
@@ -201,10 +206,9 @@ __device__ __forceinline__ void masked_acc_unit(const GemmParams& p, uint32_t st
                           __float_as_uint(__uint_as_float(y[c][pass].y) + add[1]),
                           __float_as_uint(__uint_as_float(y[c][pass].z) + add[2]),
                           __float_as_uint(__uint_as_float(y[c][pass].w) + add[3]));
-        o[1] = make_uint4(__float_as_uint(__uint_as_float(y2[c][pass].x) + add[4]),
-                          __float_as_uint(__uint_as_float(y2[c][pass].y) + add[5]),
-                          __float_as_uint(__uint_as_float(y2[c][pass].z) + add[6]),
-                          __float_as_uint(__uint_as_float(y2[c][pass].w) + add[7]));
+        const uint4 z = y2[f32 ? c : 0][pass];
+        o[1] = make_uint4(__float_as_uint(__uint_as_float(z.x) + add[4]), __float_as_uint(__uint_as_float(z.y) + add[5]),
+                          __float_as_uint(__uint_as_float(z.z) + add[6]), __float_as_uint(__uint_as_float(z.w) + add[7]));
       } else {
         const uint32_t yy[4] = {y[c][pass].x, y[c][pass].y, y[c][pass].z, y[c][pass].w};
         uint32_t w[4];
@@ -370,12 +374,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 2 + 4 * C::EpiGroups) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int eg = (warp - 2) >> 2;         // with two groups: the accumulator buffer this group drains
     int acc = 0;
     uint32_t aph = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      if (C::EpiGroups == 2 && acc != eg) {
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+        continue;
+      }
       int mb, nb, split, kt0, nmain, next;
       decode_unit(p, u, mb, nb, split, kt0, nmain, next);
       if (!mbar_wait(&acc_full[acc], aph)) break;
@@ -383,7 +393,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       const int row = mb * 128 + q * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
       if (p.out_mode == kOutMaskAccBF16 || p.out_mode == kOutMaskAccF32) {
-        masked_acc_unit<C::BN / 32>(p, smem_u32(sEpi + q * 4096), lane, mb * 128 + q * 32, nb * C::BN, t_row);
+        if (p.out_mode == kOutMaskAccF32) {   // fp32 dX: two round trips of half the columns (registers)
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h)
+            masked_acc_unit<C::BN / 64, true>(p, smem_u32(sEpi + (warp - 2) * 4096), lane, mb * 128 + q * 32,
+                                              nb * C::BN + h * (C::BN / 2), t_row + h * (C::BN / 2));
+        } else
+          masked_acc_unit<C::BN / 32, false>(p, smem_u32(sEpi + (warp - 2) * 4096), lane, mb * 128 + q * 32,
+                                             nb * C::BN, t_row);
       } else {
 #pragma unroll 1
         for (int c = 0; c < C::BN / 32; ++c) {
@@ -469,10 +486,11 @@ using CfgGrad = GemmCfg<64, 6, true, kB_TmaMN, false, true>;
 using CfgDownK128 = GemmCfg<128, 5, false, kB_TmaK, false, false>;
 using CfgDownMN128 = GemmCfg<128, 5, false, kB_TmaMN, false, false>;
 using CfgGrad128 = GemmCfg<128, 4, true, kB_TmaMN, false, true>;
+using CfgUpMasked = GemmCfg<128, 4, false, kB_TmaMN, false, false, 2>;
 
 int gemm_bn(GemmKind kind) {
   switch (kind) {
-    case kGemmLoraDownK128: case kGemmLoraDownMN128: case kGemmLoraGrad128: return 128;
+    case kGemmLoraDownK128: case kGemmLoraDownMN128: case kGemmLoraGrad128: case kGemmLoraUpMasked: return 128;
     default: return 64;
   }
 }
@@ -486,6 +504,7 @@ static cudaError_t launch_gemm_impl(GemmKind kind, const GemmParams& p, const Ge
     case kGemmLoraDownK128: return launch_cfg<CfgDownK128>(p, maps, grid, st);
     case kGemmLoraDownMN128: return launch_cfg<CfgDownMN128>(p, maps, grid, st);
     case kGemmLoraGrad128: return launch_cfg<CfgGrad128>(p, maps, grid, st);
+    case kGemmLoraUpMasked: return launch_cfg<CfgUpMasked>(p, maps, grid, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -387,8 +387,9 @@ int run_lora_up_masked(const Plan& P, const uint16_t* sG, int64_t m, int64_t k, 
   Split sp;
   sp.splits = 1;
   sp.kps = P.r_pad / 64;
-  // 128-column tiles: each epilogue warp fetches 32 rows x 128 columns of dX in one round trip
-  GemmParams p = base_params(m, k, gemm_bn(kGemmLoraDownMN128), P.r_pad / 64, sp);
+  // 128-column tiles: each epilogue warp fetches 32 rows x 128 columns of dX in one round trip, and two
+  // epilogue groups keep two units' round trips in flight
+  GemmParams p = base_params(m, k, gemm_bn(kGemmLoraUpMasked), P.r_pad / 64, sp);
   p.out = dX;
   p.ld_out = k;
   p.out_mode = dx_f32 ? kOutMaskAccF32 : kOutMaskAccBF16;
@@ -399,7 +400,7 @@ int run_lora_up_masked(const Plan& P, const uint16_t* sG, int64_t m, int64_t k, 
   bool ok = map_bf16(&maps.a, sG, m, P.r_pad, 128);                              // [m, r_pad], K-major
   ok = ok && tmap_2d(&maps.b, A, kBF16, k, r, k * 2, 64, 64, 128);                 // A [r, k]: MN-major
   if (!ok) return QLORA_ERR_CUDA;
-  return cuda_status(launch_gemm(kGemmLoraDownMN128, p, maps, grid_of(p), st));
+  return cuda_status(launch_gemm(kGemmLoraUpMasked, p, maps, grid_of(p), st));
 }
 
 // dB (rows = n, act = dY) or dA^T (rows = k, act = X): sum over tokens of act^T . [hi + lo].

@@ -94,6 +94,7 @@ enum GemmKind : int {
   kGemmLoraDownK128 = 5,
   kGemmLoraDownMN128 = 6,
   kGemmLoraGrad128 = 7,
+  kGemmLoraUpMasked = 8,   // as kGemmLoraDownMN128 (K = rank), two epilogue groups: dropout's masked dX term
 };
 
 int gemm_bn(GemmKind kind);
