@@ -50,9 +50,6 @@ struct WCfg {
   static constexpr int kATile = 128 * 64 * 2;
   static constexpr int kBTile = TOK * 64 * 2;
   static constexpr int kRBytes = 4096;      // packed codes of one 128 x 64 weight tile
-  // K steps of packed codes the producer hints into L2 ahead of its loads: at few tokens
-  // the ring holds too few bytes to cover the DRAM latency of the weight stream
-  static constexpr int kPrefetch = (kBN <= 16) ? 24 : 0;
   static constexpr int kThreads = (6 + 4 * (kGroups >= 2 ? kGroups : 2)) * 32;
   static constexpr int kAccBufs = (2 * TOK <= 512) ? 2 : 1;   // double-buffer the accumulators when TMEM allows
   static constexpr int kTmemCols = (kAccBufs * TOK <= 32) ? 32 : (kAccBufs * TOK <= 64) ? 64 : (kAccBufs * TOK <= 128) ? 128
@@ -216,15 +213,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         int mb, nb, split, kt0, nmain, next;
         wdecode(p, u, mb, nb, split, kt0, nmain, next);
-        auto prefetch_codes = [&](int i) {
-          if (C::Bwd) tma_prefetch_l2_2d(&maps.codes, mb * 64, (kt0 + i) * 64);
-          else tma_prefetch_l2_2d(&maps.codes, (kt0 + i) * 32, mb * 128);
-        };
-        if (C::kPrefetch > 0)
-          for (int j = C::Stages; j < C::kPrefetch && j < nmain; ++j) prefetch_codes(j);
         for (int i = 0; i < nmain + next; ++i) {
-          if (C::kPrefetch > 0 && i + C::kPrefetch < nmain && i + C::kPrefetch >= C::Stages)
-            prefetch_codes(i + C::kPrefetch);
           if (!mbar_wait(&empty[stage], ph ^ 1)) { ok = false; break; }
           uint64_t* bar = &tma_full[stage];
           uint8_t* a_dst = sA + stage * C::kATile;
