@@ -1,6 +1,7 @@
 // Small memory-bound kernels around the tensor-core GEMMs: split reductions
 // of the low-rank products, hi/lo bf16 splitting, gradient finalisation and
 // the SiLU-gated glue between the MLP projections.
+#include <cstring>
 #include "qlora_kernels.h"
 
 namespace qlora {
@@ -163,42 +164,59 @@ cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_str
 
 // ---------------------------------------------------------------------------
 // U = X A^T for a few tokens on CUDA cores (the tensor-core path would pad the
-// 128-row tile with mostly empty rows). Grid (adapter row j, K slice of 1024):
-// each thread takes 8 consecutive K of its slice for every token, a block
-// reduction gives the slice's partial, and lora_finalize_kernel sums the
-// slices in a fixed order.
+// 128-row tile with mostly empty rows), finished in the same launch. A cluster of
+// eight CTAs per adapter row j splits K into eight slices: each thread takes 8
+// consecutive K at a stride of 1024 within its slice for every token, a fixed-order
+// block reduction gives the slice's partial, and the cluster's first CTA adds the
+// eight partials in slice order through distributed shared memory. It writes U
+// (fp32, optional) and bf16(scale * U) for the forward's K extension; rows j >= r
+// of the padded operand get zeros.
 // ---------------------------------------------------------------------------
-constexpr int kSmallSlice = 1024;
+constexpr int kSmallThreads = 128;
+constexpr int kSmallSlices = 8;     // CTAs per cluster (portable cluster size)
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
 
 template <int MMAX>
-__global__ void __launch_bounds__(128) lora_down_small_kernel(const uint16_t* __restrict__ X, int m, int64_t k,
-                                                              const uint16_t* __restrict__ A, int r_pad,
-                                                              float* __restrict__ part) {
-  __shared__ float red[4][MMAX];
-  const int j = blockIdx.x;
-  const int ks = blockIdx.y;
-  const int64_t kk = static_cast<int64_t>(ks) * kSmallSlice + threadIdx.x * 8;
+__global__ void __launch_bounds__(kSmallThreads) lora_down_small_kernel(const uint16_t* __restrict__ X, int m,
+                                                                       int64_t k, const uint16_t* __restrict__ A,
+                                                                       int r, int r_pad, float scale, float pre,
+                                                                       float* __restrict__ out_f32,
+                                                                       uint16_t* __restrict__ out_scaled) {
+  __shared__ float red[kSmallThreads / 32][MMAX];
+  __shared__ float slice_sum[MMAX];
+  const int j = blockIdx.x / kSmallSlices;
+  const uint32_t slice = cluster_ctarank();
+  const int64_t slice_len = ((k / 8 + kSmallSlices - 1) / kSmallSlices) * 8;
+  const int64_t k0 = static_cast<int64_t>(slice) * slice_len;
+  const int64_t k1 = (k0 + slice_len < k) ? k0 + slice_len : k;
   float acc[MMAX];
 #pragma unroll
   for (int i = 0; i < MMAX; ++i) acc[i] = 0.f;
-  if (kk < k) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * k + kk));
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    float af[8];
+  if (j < r) {
+    for (int64_t kk = k0 + static_cast<int64_t>(threadIdx.x) * 8; kk < k1; kk += kSmallThreads * 8) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * k + kk));
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+      float af[8];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      af[2 * t] = __uint_as_float(aw[t] << 16);
-      af[2 * t + 1] = __uint_as_float(aw[t] & 0xFFFF0000u);
-    }
+      for (int t = 0; t < 4; ++t) {
+        af[2 * t] = __uint_as_float(aw[t] << 16);
+        af[2 * t + 1] = __uint_as_float(aw[t] & 0xFFFF0000u);
+      }
 #pragma unroll
-    for (int i = 0; i < MMAX; ++i) {
-      if (i < m) {
-        const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(i) * k + kk));
-        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+      for (int i = 0; i < MMAX; ++i) {
+        if (i < m) {
+          const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(i) * k + kk));
+          const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          acc[i] = fmaf(__uint_as_float(xw[t] << 16), af[2 * t], acc[i]);
-          acc[i] = fmaf(__uint_as_float(xw[t] & 0xFFFF0000u), af[2 * t + 1], acc[i]);
+          for (int t = 0; t < 4; ++t) {
+            acc[i] = fmaf(__uint_as_float(xw[t] << 16), af[2 * t], acc[i]);
+            acc[i] = fmaf(__uint_as_float(xw[t] & 0xFFFF0000u), af[2 * t + 1], acc[i]);
+          }
         }
       }
     }
@@ -212,25 +230,49 @@ __global__ void __launch_bounds__(128) lora_down_small_kernel(const uint16_t* __
     if (lane == 0) red[warp][i] = v;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < m; i += blockDim.x)
-    part[(static_cast<int64_t>(ks) * m + i) * r_pad + j] = red[0][i] + red[1][i] + red[2][i] + red[3][i];
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSmallThreads / 32; ++w) v += red[w][i];
+    slice_sum[i] = v;
+  }
+  cluster_sync();                          // every slice's partial is in its CTA's shared memory
+  if (slice == 0) {
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+      float u = 0.f;
+      for (uint32_t t = 0; t < kSmallSlices; ++t) u += ld_shared_cluster_f32(smem_cluster_addr(&slice_sum[i], t));
+      u = __fmul_rn(pre, u);
+      if (out_f32 != nullptr && j < r) out_f32[static_cast<int64_t>(i) * r + j] = u;
+      out_scaled[static_cast<int64_t>(i) * r_pad + j] = f2bf(__fmul_rn(scale, u));
+    }
+  }
+  cluster_sync();                          // no CTA leaves while the first one still reads its partial
 }
 
-int lora_down_small_slices(int64_t k) { return static_cast<int>((k + kSmallSlice - 1) / kSmallSlice); }
-
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
-                                   int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
-                                   cudaStream_t st, float pre) {
-  const int ks = lora_down_small_slices(k);
-  const dim3 grid(static_cast<unsigned>(r), static_cast<unsigned>(ks));
-  if (m <= 16)
-    lora_down_small_kernel<16><<<grid, 128, 0, st>>>(X, static_cast<int>(m), k, A, r_pad, part);
-  else
-    lora_down_small_kernel<64><<<grid, 128, 0, st>>>(X, static_cast<int>(m), k, A, r_pad, part);
+                                   int32_t r_pad, float scale, float* U32, uint16_t* sU, cudaStream_t st, float pre) {
+  if (m > 64 || k % 8 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(r_pad * kSmallSlices), 1, 1);
+  cfg.blockDim = dim3(kSmallThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSmallSlices;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int mi = static_cast<int>(m);
+  cudaError_t e = (m <= 16)
+                      ? cudaLaunchKernelEx(&cfg, lora_down_small_kernel<16>, X, mi, k, A, static_cast<int>(r),
+                                           static_cast<int>(r_pad), scale, pre, U32, sU)
+                      : cudaLaunchKernelEx(&cfg, lora_down_small_kernel<64>, X, mi, k, A, static_cast<int>(r),
+                                           static_cast<int>(r_pad), scale, pre, U32, sU);
   count_launches(1);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_lora_finalize(part, ks, m * r_pad, m, r, r_pad, scale, U32, sU, nullptr, nullptr, st, pre);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------

@@ -45,6 +45,7 @@ __device__ int g_device_error = 0;
 // ---------------------------------------------------------------------------
 constexpr int kQChunk = 128;     // 64-blocks per chunk: 32 KB of fp32 weights
 constexpr int kQStages = 3;
+constexpr int kQCtasPerSm = 2;    // resident CTAs per SM (shared memory: kQStages stages each)
 constexpr int kQStage = kQChunk * 256;                // bytes per stage: two 16 KB boxes of half-blocks
 constexpr int kQSmem = kQStages * kQStage + 1024;     // + alignment of the swizzled stages
 
@@ -131,7 +132,7 @@ __device__ double tree_sum_cta(const double* __restrict__ part, int64_t n, doubl
 }
 
 template <bool kDQ>
-__global__ void __launch_bounds__(256, 2) nf4_quantize_kernel(const __grid_constant__ CUtensorMap wmap,
+__global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __grid_constant__ CUtensorMap wmap,
                                                               const float* __restrict__ W, int64_t n_elem,
                                                               Nf4Buckets bk, uint8_t* __restrict__ codes,
                                                               uint16_t* __restrict__ scale_bf16,
@@ -457,7 +458,8 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   const int64_t nblk = (n_elem + 63) / 64;
   const bool dq = (scale_fp8 != nullptr);
   const int64_t nchunks = (nblk + kQChunk - 1) / kQChunk;
-  const int grid = static_cast<int>(nchunks < 2LL * num_sms ? nchunks : 2LL * num_sms);
+  const int64_t slots = static_cast<int64_t>(kQCtasPerSm) * num_sms;
+  const int grid = static_cast<int>(nchunks < slots ? nchunks : slots);
   // W as rows of one 64-block; boxes of 128 rows x 32 floats (128 B, swizzled)
   CUtensorMap wmap;
   std::memset(&wmap, 0, sizeof(wmap));

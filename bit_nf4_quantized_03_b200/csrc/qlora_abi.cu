@@ -273,7 +273,6 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   part = std::max(part, static_cast<size_t>(P.db.splits) * n * rp);
   part = std::max(part, static_cast<size_t>(P.da.splits) * k * rp);
   if (P.fwd.splits > 1) part = std::max(part, static_cast<size_t>(P.fwd.splits) * m * n);
-  if (m <= 64) part = std::max(part, static_cast<size_t>(lora_down_small_slices(k)) * m * rp);
   // dX through fp32 partials: for split K, and for an accumulating dX on the CTA-pair path
   if (P.bwd.splits > 1 || wrows == 256)
     part = std::max(part, static_cast<size_t>(std::max(P.bwd.splits, 1)) * m * k);
@@ -558,8 +557,7 @@ int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m,
 
   // U = c (M * X) A^T (fp32, optionally saved) and bf16(s * U) for the K extension
   if (m <= 64) {
-    if (launch_lora_down_small(Xl, m, k, A, r, P.r_pad, s, U_save, sU, reinterpret_cast<float*>(wsb + P.off_part),
-                               st, D.keep) != cudaSuccess)
+    if (launch_lora_down_small(Xl, m, k, A, r, P.r_pad, s, U_save, sU, st, D.keep) != cudaSuccess)
       return QLORA_ERR_CUDA;
   } else {
     const int rc = run_lora_down(P, false, Xl, m, k, A, r, s, wsb, U_save, sU, nullptr, nullptr, st, D.keep);

@@ -160,13 +160,12 @@ cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_str
 cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_stride, int64_t rows,
                                  int64_t cols, int64_t ld_part, void* out, int out_bf16, int accumulate,
                                  cudaStream_t st);
-// U = X A^T on CUDA cores for a few tokens (m <= 64): fp32 U [m, r] (nullable) and
-// bf16(scale * U) [m, r_pad] (padding columns zeroed), via K-slice partials.
-// part: workspace of lora_down_small_slices(k) * m * r_pad floats for the K-slice partials.
-int lora_down_small_slices(int64_t k);
+// U = X A^T on CUDA cores for a few tokens (m <= 64, k % 8 == 0), one launch, no
+// workspace: fp32 pre * U [m, r] (nullable) and bf16(scale * pre * U) [m, r_pad]
+// (padding columns zeroed).
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
-                                   int32_t r_pad, float scale, float* U32, uint16_t* sU, float* part,
-                                   cudaStream_t st, float pre = 1.0f);
+                                   int32_t r_pad, float scale, float* U32, uint16_t* sU, cudaStream_t st,
+                                   float pre = 1.0f);
 // LoRA dropout (dropout.cu): keep mask from Philox4x32-10, masked copy of X, packed mask bits.
 cudaError_t launch_dropout_mask(const uint16_t* X, int64_t count, uint32_t thr, uint64_t seed, uint64_t offset,
                                 uint16_t* Xd, uint8_t* mask, cudaStream_t st);
