@@ -46,6 +46,8 @@ def test_single_linear_256_r8():
     (130, 512, 384, 128),
     (1, 256, 256, 64),       # single token
     (16, 1024, 2048, 64),    # small-M split-K path
+    (40, 512, 832, 32),      # 17-64 tokens: the wider small-M U kernel; K slices of 104, padded rank rows
+    (8, 256, 512, 8),        # rank 8 padded to 64 in the forward's K extension
     (72, 4096, 1024, 16),
 ])
 def test_linear_shapes_and_ranks(m, n, k, r):
