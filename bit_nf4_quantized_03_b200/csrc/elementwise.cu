@@ -170,7 +170,8 @@ cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_str
 // block reduction gives the slice's partial, and the cluster's first CTA adds the
 // eight partials in slice order through distributed shared memory. It writes U
 // (fp32, optional) and bf16(scale * U) for the forward's K extension; rows j >= r
-// of the padded operand get zeros.
+// of the padded operand get zeros. The fused GEMM that follows may be launched to
+// start early and overlap this kernel (it waits before reading bf16(scale * U)).
 // ---------------------------------------------------------------------------
 constexpr int kSmallThreads = 128;
 constexpr int kSmallSlices = 8;     // CTAs per cluster (portable cluster size)
@@ -189,6 +190,9 @@ __global__ void __launch_bounds__(kSmallThreads) lora_down_small_kernel(const ui
                                                                        uint16_t* __restrict__ out_scaled) {
   __shared__ float red[kSmallThreads / 32][MMAX];
   __shared__ float slice_sum[MMAX];
+  // the fused GEMM launched after this kernel may start streaming its weight now; it
+  // waits for this grid before it reads bf16(scale * U)
+  griddep_launch_dependents();
   const int j = blockIdx.x / kSmallSlices;
   const uint32_t slice = cluster_ctarank();
   const int64_t slice_len = ((k / 8 + kSmallSlices - 1) / kSmallSlices) * 8;

@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       uint32_t ph = 0;
       uint32_t pending = 0, pend_par = 0;
       bool ok = true;
+      bool ext_ready = false;   // the low-rank operand (s*U or s*G) of the previous launch is visible
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         int mb, nb, split, kt0, nmain, next;
         wdecode(p, u, mb, nb, split, kt0, nmain, next);
@@ -218,6 +219,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           uint64_t* bar = &tma_full[stage];
           uint8_t* a_dst = sA + stage * C::kATile;
           uint8_t* b_dst = sB + stage * C::kBTile;
+          if (i >= nmain && !ext_ready) {
+            // a launch that may start early (programmatic dependent launch) streams the weight
+            // while the kernel that writes the low-rank operand finishes; wait here, before the
+            // first load of that operand (a no-op for an ordinary launch)
+            griddep_wait();
+            ext_ready = true;
+          }
           if (i < nmain) {
             const int kt = kt0 + i;
             mbar_arrive_expect_tx(bar, C::kRBytes + C::kBTile);
@@ -940,7 +948,7 @@ int wgemm_pair_slots() {
 }
 
 template <class C>
-static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st) {
+static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st, bool early) {
   static bool attr_set[64] = {};
   static std::mutex mu;
   int dev = 0;
@@ -955,8 +963,22 @@ static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid,
       attr_set[dev] = true;
     }
   }
-  qlora_wgemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p, maps);
-  return cudaGetLastError();
+  if (!early) {
+    qlora_wgemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p, maps);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qlora_wgemm_kernel<C>, p, maps);
 }
 
 int wgemm_box_rows(int bn) { return bn >= 256 ? 128 : bn; }   // a CTA pair loads half of each 256-token tile
@@ -978,7 +1000,7 @@ int wgemm_bn(int64_t tokens) {
 }
 
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
-                         double algo_flops) {
+                         double algo_flops, bool early) {
   // the tile counts must be those of the kernel this width selects
   if (p.tiles_n != (static_cast<int64_t>(p.cols) + bn - 1) / bn ||
       p.tiles_m != (static_cast<int64_t>(p.rows) + wgemm_tile_rows(bn) - 1) / wgemm_tile_rows(bn))
@@ -988,17 +1010,17 @@ cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& map
   cudaError_t e = cudaErrorInvalidValue;
   if (!bwd) {
     switch (bn) {
-      case 16: e = launch_wcfg<WCfg<16, 1, 9, false, 3>>(p, maps, grid, st); break;
-      case 64: e = launch_wcfg<WCfg<64, 1, 6, false, 3>>(p, maps, grid, st); break;
-      case 128: e = launch_wcfg<WCfg<128, 1, 6, false, 3>>(p, maps, grid, st); break;
+      case 16: e = launch_wcfg<WCfg<16, 1, 9, false, 3>>(p, maps, grid, st, early); break;
+      case 64: e = launch_wcfg<WCfg<64, 1, 6, false, 3>>(p, maps, grid, st, early); break;
+      case 128: e = launch_wcfg<WCfg<128, 1, 6, false, 3>>(p, maps, grid, st, early); break;
       case 256: e = launch_pcfg<PCfg<6, false, 2, 1>>(p, maps, grid, st); break;   // CTA pair
       case 512: e = launch_pcfg<PCfg<4, false, 2, 2>>(p, maps, grid, st); break;   // CTA pair, two token tiles
     }
   } else {
     switch (bn) {
-      case 16: e = launch_wcfg<WCfg<16, 1, 9, true, 3>>(p, maps, grid, st); break;
-      case 64: e = launch_wcfg<WCfg<64, 1, 6, true, 3>>(p, maps, grid, st); break;
-      case 128: e = launch_wcfg<WCfg<128, 1, 6, true, 3>>(p, maps, grid, st); break;
+      case 16: e = launch_wcfg<WCfg<16, 1, 9, true, 3>>(p, maps, grid, st, early); break;
+      case 64: e = launch_wcfg<WCfg<64, 1, 6, true, 3>>(p, maps, grid, st, early); break;
+      case 128: e = launch_wcfg<WCfg<128, 1, 6, true, 3>>(p, maps, grid, st, early); break;
       case 256: e = launch_pcfg<PCfg<6, true, 2, 1>>(p, maps, grid, st); break;    // CTA pair
       case 512: e = launch_pcfg<PCfg<4, true, 2, 2>>(p, maps, grid, st); break;    // CTA pair, two token tiles
     }

@@ -589,7 +589,9 @@ int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m,
   ok = ok && map_bf16(&maps.b2, sU, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
   if (!ok) return QLORA_ERR_CUDA;
   const double fwd_flops = 2.0 * double(m) * double(n) * double(k + r);
-  cudaError_t e = launch_wgemm(false, P.bn, p, maps, wgemm_grid(p, P.bn, num_sms()), st, fwd_flops);
+  // at few tokens U comes from lora_down_small_kernel right before: the GEMM may start streaming
+  // the weight while that kernel runs, and waits for it before its K extension
+  cudaError_t e = launch_wgemm(false, P.bn, p, maps, wgemm_grid(p, P.bn, num_sms()), st, fwd_flops, m <= 64);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   if (P.fwd.splits > 1) {
     e = launch_splitk_reduce(static_cast<const float*>(p.out), P.fwd.splits, p.part_stride, m, n, n, Y,

@@ -137,6 +137,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. griddep_wait: block until the grids this one was
+// launched after have completed and their writes are visible (returns at once when
+// the launch did not allow an early start). griddep_launch_dependents: from this CTA's
+// side, a grid launched after this one with that allowance may start now.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y) {
   asm volatile(

@@ -122,8 +122,12 @@ int wgemm_box_rows(int bn);              // token rows per TMA box (each CTA of 
 int wgemm_tile_rows(int bn);             // weight rows per tile: 256 when a CTA pair shares it
 int wgemm_pair_slots();                  // CTA pairs resident at once
 int wgemm_grid(const GemmParams& p, int bn, int sms);   // CTAs to launch (even for CTA pairs)
+// early: the single-CTA kernel (bn <= 128) may start before the preceding kernel on the
+// stream has finished (programmatic dependent launch); it waits for that kernel only
+// before its first load of the low-rank operand, which that kernel must write and
+// nothing else it reads or writes. Ignored by the CTA-pair kernel.
 cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& maps, int grid, cudaStream_t st,
-                         double algo_flops);
+                         double algo_flops, bool early = false);
 
 // ---------------------------------------------------------- adapter merge
 // (nf4_merge.cu) out[n, k] = dequant(W) + scale * B . A, tiles of 128 rows x
