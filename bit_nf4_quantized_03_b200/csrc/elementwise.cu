@@ -256,8 +256,7 @@ __global__ void __launch_bounds__(kSmallThreads) lora_down_small_kernel(const ui
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
                                    int32_t r_pad, float scale, float* U32, uint16_t* sU, cudaStream_t st, float pre) {
   if (m > 64 || k % 8 != 0) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(r_pad * kSmallSlices), 1, 1);
   cfg.blockDim = dim3(kSmallThreads, 1, 1);
   cfg.stream = st;

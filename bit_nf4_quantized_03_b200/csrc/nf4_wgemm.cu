@@ -896,8 +896,7 @@ static cudaError_t launch_pcfg(const GemmParams& p, const WMaps& maps, int grid,
     }
   }
   if (grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
@@ -926,8 +925,7 @@ int wgemm_pair_slots() {
   int slots = sms / 2;
   if (cudaFuncSetAttribute(qlora_wgemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes) == cudaSuccess) {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(C::kThreads, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
@@ -967,8 +965,7 @@ static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid,
     qlora_wgemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p, maps);
     return cudaGetLastError();
   }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;

@@ -281,7 +281,7 @@ Plan make_plan(int64_t m, int64_t n, int64_t k, int32_t r) {
   return P;
 }
 
-bool linear_args_ok(const qlora_nf4_weight* w, const void* X, int64_t m, const void* A, const void* B, int32_t r) {
+bool linear_args_ok(const qlora_nf4_weight* w, const void* X, int64_t m, const void* A, const void* B) {
   if (!weight_ok(w) || X == nullptr || A == nullptr || B == nullptr) return false;
   if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return false;
   if (m < 1 || m > (int64_t(1) << 31) - 1) return false;
@@ -531,7 +531,7 @@ int qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, co
 int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m, const uint16_t* A,
                         const uint16_t* B, int32_t r, float alpha, void* Y, int32_t y_dtype, float* U_save,
                         const qlora_dropout* drop, void* ws, size_t ws_bytes, qlora_stream_t stream) {
-  if (!linear_args_ok(w, X, m, A, B, r) || Y == nullptr || !aligned16(Y)) return QLORA_ERR_INVALID;
+  if (!linear_args_ok(w, X, m, A, B) || Y == nullptr || !aligned16(Y)) return QLORA_ERR_INVALID;
   if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_FP32) return QLORA_ERR_INVALID;
   if (U_save != nullptr && !aligned16(U_save)) return QLORA_ERR_INVALID;
   const int sst = linear_shape_status(w, r);
@@ -612,7 +612,7 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
                         const uint16_t* A, const uint16_t* B, int32_t r, float alpha, const float* U_saved,
                         void* dX, int32_t dx_dtype, float* dA, float* dB, int32_t flags, const qlora_dropout* drop,
                         void* ws, size_t ws_bytes, qlora_stream_t stream) {
-  if (!linear_args_ok(w, X, m, A, B, r) || dY == nullptr || !aligned16(dY)) return QLORA_ERR_INVALID;
+  if (!linear_args_ok(w, X, m, A, B) || dY == nullptr || !aligned16(dY)) return QLORA_ERR_INVALID;
   if (dA == nullptr || dB == nullptr || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_INVALID;
   if (dX != nullptr && (!aligned16(dX) || (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_FP32)))
     return QLORA_ERR_INVALID;
