@@ -115,52 +115,89 @@ def all_reduce_grads(flat) -> None:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs.
+    The sampler is started, and its first sample awaited, before the region; each
+    sample carries nvidia-smi's timestamp, and only those stamped inside the region
+    (plus one interval after it, which still reports the region's last moments)
+    are summarised."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.first = ""
+        self.out = ""
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
-                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
-                                         stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", str(self.INTERVAL_MS), "-i", str(self.dev)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
+        if self.proc is not None:
+            try:
+                import select
+                ready, _, _ = select.select([self.proc.stdout], [], [], 5.0)
+                if ready:
+                    self.first = self.proc.stdout.readline()
+            except (OSError, ValueError):
+                pass
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *a):
-        self.out = ""
+        self.t1 = time.time()
+        rest = ""
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(2.0 * self.INTERVAL_MS / 1000.0)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                rest, _ = self.proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                rest, _ = self.proc.communicate()
+        self.out = (self.first or "") + (rest or "")
+
+    @staticmethod
+    def _stamp(text: str):
+        import datetime
+        try:
+            return datetime.datetime.strptime(text.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def summary(self) -> dict:
-        sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in (self.out or "").splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1].split()[0]))
-                smax = float(parts[2].split()[0])
-            except ValueError:
+                sm = float(parts[2].split()[0])
+                smax = float(parts[3].split()[0])
+            except (ValueError, IndexError):
                 continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            active = {nm for nm, v in zip(names, parts[6:10]) if v.lower().startswith("active")}
+            rows.append((self._stamp(parts[0]), sm, smax, active))
+        window = "timed region"
+        if self.t0 is not None and self.t1 is not None:
+            late = self.t1 + self.INTERVAL_MS / 1000.0
+            inside = [r for r in rows if r[0] is not None and self.t0 <= r[0] <= late]
+        else:
+            inside = []
+        if not inside:             # region shorter than the sampling interval, or no timestamps
+            inside, window = rows, "all samples"
+        sm = [r[1] for r in inside]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": inside[-1][2] if inside else None,
+                "reasons": sorted(set().union(*[r[3] for r in inside])) if inside else [],
+                "samples": len(sm), "window": window}
 
 
 def blas_threads() -> int:
