@@ -24,8 +24,8 @@ Readings taken where the pages are silent or garbled (each is listed in the
 design notes of the repository):
 
 1. Levels: the pages say 16 levels at quantiles of a normal distribution
-   ([CSD] NF4 section, [GAMUT] NF4 section); the benchmark spec adds an
-   exact zero and normalisation to [-1, 1]. We take the asymmetric quantile
+   ([CSD] NF4 section, [GAMUT] NF4 section), with an exact zero and
+   normalisation to [-1, 1] (the format's definition here). We take the asymmetric quantile
    construction of the NF4 paper: 8 positive quantiles Phi^-1(p) at p
    equally spaced from delta down to 1/2 (9 points, 1/2 dropped), 7
    negative ones built the same way on 8 points, plus an exact 0, all
@@ -39,10 +39,10 @@ design notes of the repository):
 4. Packing: byte j holds element 2j in its low nibble and 2j+1 in its high
    nibble; an odd tail leaves the high nibble 0.
 5. Plain scale: bf16 (round to nearest even) of the fp32 absmax ([CSD]
-   worked example: "one scale factor ... in BF16").
-6. Double quantization ([CSD] DQ section says "8-bit FP8 blocks"; the block
-   of 256, the fp32 second-level scale and the mean offset come from the
-   task statement): mu = fp32(S / nblk) with S the fp64 sum of all absmax
+   worked example, where each block keeps a single BF16 scale).
+6. Double quantization ([CSD] DQ section: the scales become 8-bit floats
+   in blocks; the block of 256, the fp32 second-level scale and the mean
+   offset are the format's definition here, the pages leaving them open): mu = fp32(S / nblk) with S the fp64 sum of all absmax
    values in a fixed pairwise order; per 256-block d = fp32(a - mu),
    s2 = fp32(max|d| / 448) (1 if max|d| = 0), q = E4M3(fp32(d / s2)) with
    round-to-nearest-even and saturation to +-448 (OCP E4M3, the FP8 whose
@@ -88,7 +88,7 @@ import numpy as np
 from scipy.special import ndtri
 
 BLOCKSIZE = 64          # [CSD] Piece 2 and NF4 section: blocks of 64 weights
-DQ_BLOCKSIZE = 256      # second-level block (task statement)
+DQ_BLOCKSIZE = 256      # second-level block (the format's definition; the pages leave it open)
 E4M3_MAX = 448.0        # largest finite OCP E4M3 value
 FLT_MIN = np.float32(np.finfo(np.float32).tiny)
 
@@ -323,7 +323,8 @@ def dequantize_f64(qw: dict, shape) -> np.ndarray:
 
 # ----------------------------------------------------------------------------
 # The frozen-base linear layer with its low-rank branch (fp64)
-# ([CSD] Piece 2 and Piece 3; the formula itself is the benchmark spec's)
+# ([CSD] Piece 2 and Piece 3, which keep the LoRA math unchanged; the formula is
+# the standard LoRA one with scale alpha / r)
 # ----------------------------------------------------------------------------
 def _f64(t) -> np.ndarray:
     """bf16/fp32 torch tensor or numpy array -> fp64 numpy (exact)."""
