@@ -97,21 +97,8 @@ def measured_peaks() -> dict:
 
 
 def max_over_ranks(x: float) -> float:
-    import torch
-    import torch.distributed as dist
-    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
-        return x
-    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def all_reduce_grads(flat) -> None:
-    """Data-parallel exchange: sum the adapter gradients of every rank."""
-    import torch.distributed as dist
-    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
-        dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+    from bit_nf4_quantized_03_b200 import dp
+    return dp.max_over_ranks(x)
 
 
 class ClockSampler:
@@ -310,13 +297,9 @@ class Workload:
         self.U = {nm: e(M, RANK_R, dt=f32) for nm, _, _ in LAYERS}
         self.y16 = {nm: e(M_SMALL, n) for nm, n, _ in LAYERS}
         # adapter gradients live in one flat buffer (one all-reduce for the data-parallel exchange)
-        sizes = [RANK_R * k + n * RANK_R for _, n, k in LAYERS]
-        self.grads = torch.zeros(sum(sizes), dtype=f32, device=dev)
-        self.dA, self.dB, o_ = {}, {}, 0
-        for (nm, n, k), sz in zip(LAYERS, sizes):
-            self.dA[nm] = self.grads[o_:o_ + RANK_R * k].view(RANK_R, k)
-            self.dB[nm] = self.grads[o_ + RANK_R * k:o_ + sz].view(n, RANK_R)
-            o_ += sz
+        from bit_nf4_quantized_03_b200 import dp
+        self.adapter_grads = dp.AdapterGrads(LAYERS, RANK_R, device=dev)
+        self.grads, self.dA, self.dB = self.adapter_grads.flat, self.adapter_grads.dA, self.adapter_grads.dB
         self.host_grads = torch.empty(self.grads.shape, dtype=f32).pin_memory()
         ws = max(max(q.qlora_linear_workspace_bytes(M, n, k, RANK_R),
                      q.qlora_linear_workspace_bytes(M_SMALL, n, k, RANK_R)) for _, n, k in LAYERS)
@@ -368,7 +351,7 @@ class Workload:
         for nm, _, _ in LAYERS:
             x = d["h16"] if nm == "down_proj" else d["x16"]
             self._fwd(nm, x, self.y16[nm], None)
-        all_reduce_grads(self.grads)
+        self.adapter_grads.all_reduce()
 
     def h2d(self):
         for k_, v in self.host.items():

@@ -206,6 +206,17 @@ int qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t m, co
  * U_saved: optional fp32 [m, r] from the forward pass (NULL: recomputed).
  * flags: QLORA_BWD_ACCUMULATE_GRADS and/or QLORA_BWD_ACCUMULATE_DX.
  * Same shape rules as qlora_linear_fwd.
+ *
+ * Token-sharded data parallelism ("QLoRA Explained", Hardware Requirements by
+ * Model Size; the FAQ on one model over several GPUs): every rank holds the
+ * same weight and adapters and calls qlora_linear_fwd / qlora_linear_bwd on
+ * its own contiguous slice of the tokens (m = that slice). Y, U and dX of a
+ * slice need nothing from other ranks. dA and dB are sums over tokens, so a
+ * rank's call yields the partial sum over its slice; the full-batch gradient
+ * is the fp32 sum of the ranks' dA and dB (one all-reduce, done by the
+ * caller: the library holds no communicator). QLORA_BWD_ACCUMULATE_GRADS adds
+ * into dA, dB instead, so several slices on one rank (gradient accumulation)
+ * sum the same way before the exchange.
  */
 int qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t m,
                      const uint16_t *A, const uint16_t *B, int32_t r, float alpha, const float *U_saved,

@@ -413,6 +413,27 @@ def test_lora_merge_against_python_loops_and_the_layer():
 
 
 # ---------------------------------------------------------------- LoRA dropout
+def test_philox_known_answer_vectors():
+    # the generator's authors' published vectors pin the whole bit stream: a swapped
+    # word, a wrong multiplier or a missing key bump changes every output word
+    rows = []
+    for line in open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            rows.append([int(t, 16) for t in line.split()])
+    assert len(rows) == 3
+    for v in rows:
+        ctr, key, want = v[0:4], v[4:6], v[6:10]
+        got = o.philox4x32_10(*ctr, *key)
+        assert [int(g) for g in got] == want, [hex(int(g)) for g in got]
+    # vectorised over many counters: every lane equals the scalar call
+    c0 = np.array([rows[0][0], rows[1][0], rows[2][0]], dtype=np.uint64)
+    cs = [np.array([r[i] for r in rows], dtype=np.uint64) for i in range(1, 6)]
+    got = o.philox4x32_10(c0, *cs)
+    for j, r in enumerate(rows):
+        assert [int(g[j]) for g in got] == r[6:10]
+
+
 def test_dropout_keep_rate_and_uniformity():
     # reading 10: 16-bit values uniform on [0, 65536); kept iff >= round(p * 65536)
     n = 1 << 22
@@ -536,3 +557,19 @@ def test_adamw_zero_gradient_only_decays():
     b = o.adamw_step(p0, np.full(3, 1.0), np.zeros(3), np.zeros(3), step=1, lr=0.1)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# ----------------------------------------------------------- error metrics ---
+def test_error_metrics_hand_computed():
+    # 2 x 2 case worked by hand: ref = [[3, 0], [0, 4]] has Frobenius norm 5 and
+    # RMS sqrt(25 / 4) = 2.5; got differs by +1 at (0, 0) and -2 at (1, 1), so the
+    # error has Frobenius norm sqrt(5) and largest magnitude 2.
+    ref = np.array([[3.0, 0.0], [0.0, 4.0]])
+    got = np.array([[4.0, 0.0], [0.0, 2.0]])
+    assert o.rel_frobenius(got, ref) == pytest.approx(math.sqrt(5.0) / 5.0, rel=1e-15)
+    assert o.max_abs_over_rms(got, ref) == pytest.approx(2.0 / 2.5, rel=1e-15)
+    # identical inputs give exactly zero; a scaled copy gives the scale error
+    assert o.rel_frobenius(ref, ref) == 0.0 and o.max_abs_over_rms(ref, ref) == 0.0
+    assert o.rel_frobenius(1.5 * ref, ref) == pytest.approx(0.5, rel=1e-15)
+    # torch tensors (as the smoke check passes them) give the same numbers
+    assert o.rel_frobenius(torch.tensor(got), torch.tensor(ref)) == pytest.approx(math.sqrt(5.0) / 5.0, rel=1e-15)
