@@ -233,6 +233,67 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
+def oracle_configs() -> dict:
+    """The oracle, as it stands, timed per workload on the host cores: quantize and
+    dequantize of the 4096 x 4096 weight with outliers (both scale modes) and the
+    single 256 x 256 layer and the 7B q_proj (fwd+bwd) in full; the 7B SiLU MLP at
+    4096 tokens on 64 sampled token rows (forward and dX through the whole chain),
+    reported as measured and as a flop-rate extrapolation to the full config."""
+    from bit_nf4_quantized_03_b200 import synth
+    from oracle import nf4_oracle as o
+    res = {}
+    W = synth.weight(4096, 4096, outlier_frac=0.001).numpy()
+    ne = W.size
+    for mode, tag, scale_b in ((o.MODE_BF16, "bf16", 2.0 / 64), (o.MODE_DQ_FP8, "dq_fp8", 1.0 / 64 + 4.0 / 16384)):
+        t0 = time.perf_counter()
+        qw = o.quantize(W, mode)
+        t1 = time.perf_counter()
+        o.dequantize(qw)
+        t2 = time.perf_counter()
+        res[f"quantize_{tag}"] = {"s": t1 - t0, "gbs": ne * (4.5 + scale_b) / (t1 - t0) / 1e9, "sample": "full"}
+        res[f"dequantize_{tag}"] = {"s": t2 - t1, "gbs": ne * (2.5 + scale_b) / (t2 - t1) / 1e9, "sample": "full"}
+    for name, (m, n, k, r) in (("single_256_r8", (128, 256, 256, 8)), ("q_proj_7b", (2048, 4096, 4096, 64))):
+        Wd = o.dequantize_f64(o.quantize(synth.weight(n, k).numpy(), o.MODE_DQ_FP8), (n, k))
+        X = synth.activations(m, k)
+        A, B = synth.lora_pair(r, k, n)
+        dY = synth.grad_output(m, n)
+        t0 = time.perf_counter()
+        o.linear_forward(Wd, X, A, B, ALPHA)
+        o.linear_backward(Wd, X, dY, A, B, ALPHA)
+        dt = time.perf_counter() - t0
+        fl = linear_flops(m, n, k, r, True)
+        res[name] = {"s": dt, "tflops": fl / dt / 1e12, "tokens_per_s": m / dt, "sample": "full"}
+    # 7B MLP chain on sampled token rows: every row's forward and dX are independent of
+    # the other rows; dA, dB are sums over tokens, so the sample computes those rows' share
+    M, H, I, rows = 4096, 4096, 11008, 64
+    idx = synth.sample_rows(M, rows).numpy()
+    Wg = o.dequantize_f64(o.quantize(synth.weight(I, H, layer=41).numpy(), o.MODE_DQ_FP8), (I, H))
+    Wu = o.dequantize_f64(o.quantize(synth.weight(I, H, layer=42).numpy(), o.MODE_DQ_FP8), (I, H))
+    Wdn = o.dequantize_f64(o.quantize(synth.weight(H, I, layer=43).numpy(), o.MODE_DQ_FP8), (H, I))
+    Ag, Bg = synth.lora_pair(RANK_R, H, I, layer=41)
+    Au, Bu = synth.lora_pair(RANK_R, H, I, layer=42)
+    Ad, Bd = synth.lora_pair(RANK_R, I, H, layer=43)
+    Xs = synth.activations(M, H, layer=41).float().numpy()[idx]
+    dYs = synth.grad_output(M, H, layer=43).float().numpy()[idx]
+    t0 = time.perf_counter()
+    g, _ = o.linear_forward(Wg, Xs, Ag, Bg, ALPHA)
+    u, _ = o.linear_forward(Wu, Xs, Au, Bu, ALPHA)
+    hh = o.silu_gate_forward(g, u)
+    o.linear_forward(Wdn, hh, Ad, Bd, ALPHA)
+    dh, _, _ = o.linear_backward(Wdn, hh, dYs, Ad, Bd, ALPHA)
+    dg, du = o.silu_gate_backward(dh, g, u)
+    o.linear_backward(Wg, Xs, dg, Ag, Bg, ALPHA)
+    o.linear_backward(Wu, Xs, du, Au, Bu, ALPHA)
+    dt = time.perf_counter() - t0
+    sample_fl = (2 * linear_flops(rows, I, H, RANK_R, True) + linear_flops(rows, H, I, RANK_R, True))
+    full_fl = 2 * linear_flops(M, I, H, RANK_R, True) + linear_flops(M, H, I, RANK_R, True)
+    rate = sample_fl / dt
+    res["mlp_7b"] = {"s": dt, "tflops": rate / 1e12, "sample": f"{rows} of {M} token rows through the whole chain "
+                     "(forward, dX, and those rows' share of dA and dB)", "extrapolated_full_s": full_fl / rate,
+                     "extrapolated_tokens_per_s": M / (full_fl / rate)}
+    return res
+
+
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -519,6 +580,80 @@ def _quant_components(q, synth, torch, dev, flush, peaks, out, qn, qk, sfx):
                                          "frac": algo / ms / 1e6 / peaks["hbm_gbs"], "algo_bytes": algo}
 
 
+def _seven_b_components(q, synth, torch, dev, flush, peaks, out):
+    """7B shapes: q_proj fwd+bwd at 2048 tokens (4096 x 4096) and the SiLU-gated MLP
+    (gate/up 11008 x 4096, down 4096 x 11008) fwd+bwd at 4096 tokens, r = 64."""
+    bf, f32 = torch.bfloat16, torch.float32
+    peak = peaks.get("bf16_tflops", 1590.0)
+
+    def mk(n, k, layer):
+        W = synth.weight(n, k, layer=layer).to(dev)
+        qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+        q.qlora_nf4_quantize(W, qw)
+        a, b = synth.lora_pair(RANK_R, k, n, layer=layer)
+        return qw, a.to(dev), b.to(dev)
+
+    # config 3: 7B q_proj, X 2048 x 4096
+    M, N, K = 2048, 4096, 4096
+    qw, a, b = mk(N, K, 40)
+    X = synth.activations(M, K, layer=40).to(dev)
+    dY = synth.grad_output(M, N, layer=40).to(dev)
+    Y = torch.empty(M, N, dtype=bf, device=dev)
+    U = torch.empty(M, RANK_R, dtype=f32, device=dev)
+    dX = torch.empty(M, K, dtype=bf, device=dev)
+    dA = torch.empty(RANK_R, K, dtype=f32, device=dev)
+    dB = torch.empty(N, RANK_R, dtype=f32, device=dev)
+    ws = torch.empty(q.qlora_linear_workspace_bytes(M, N, K, RANK_R), dtype=torch.uint8, device=dev)
+
+    def qproj():
+        q.qlora_linear_fwd(qw, X, a, b, RANK_R, ALPHA, Y, q.QLORA_DTYPE_BF16, U, ws)
+        q.qlora_linear_bwd(qw, X, dY, a, b, RANK_R, ALPHA, U, dX, q.QLORA_DTYPE_BF16, dA, dB, 0, ws)
+    for _ in range(3):
+        qproj()
+    ms = graph_time(qproj, 10, flush)
+    fl = linear_flops(M, N, K, RANK_R, True)
+    out["q_proj_7b_fwd_bwd"] = {"us": ms * 1e3, "tflops": fl / ms / 1e9, "tokens_per_s": M / (ms * 1e-3),
+                                "frac_bf16_burst": fl / ms / 1e9 / peak, "flops": fl, "tokens": M}
+    del qw, X, dY, Y, U, dX, dA, dB, ws
+    # config 4: 7B MLP, 4096 tokens, gate/up 11008 x 4096, down 4096 x 11008, SiLU between
+    M, H, I = 4096, 4096, 11008
+    lay = {"gate": mk(I, H, 41), "up": mk(I, H, 42), "down": mk(H, I, 43)}
+    X = synth.activations(M, H, layer=41).to(dev)
+    dY = synth.grad_output(M, H, layer=43).to(dev)
+    e = lambda *sh, dt=bf: torch.empty(*sh, dtype=dt, device=dev)
+    g, u, h, y, dh, dg, du, dx = e(M, I), e(M, I), e(M, I), e(M, H), e(M, I), e(M, I), e(M, I), e(M, H)
+    Us = {nm: e(M, RANK_R, dt=f32) for nm in lay}
+    dAs = {nm: e(RANK_R, lay[nm][0].k, dt=f32) for nm in lay}
+    dBs = {nm: e(lay[nm][0].n, RANK_R, dt=f32) for nm in lay}
+    ws = torch.empty(max(q.qlora_linear_workspace_bytes(M, I, H, RANK_R),
+                         q.qlora_linear_workspace_bytes(M, H, I, RANK_R)), dtype=torch.uint8, device=dev)
+
+    def fwd(nm, x, yy):
+        qw_, a_, b_ = lay[nm]
+        q.qlora_linear_fwd(qw_, x, a_, b_, RANK_R, ALPHA, yy, q.QLORA_DTYPE_BF16, Us[nm], ws)
+
+    def bwd(nm, x, dy, dxx, acc):
+        qw_, a_, b_ = lay[nm]
+        q.qlora_linear_bwd(qw_, x, dy, a_, b_, RANK_R, ALPHA, Us[nm], dxx, q.QLORA_DTYPE_BF16, dAs[nm], dBs[nm],
+                           q.QLORA_BWD_ACCUMULATE_DX if acc else 0, ws)
+
+    def mlp():
+        fwd("gate", X, g)
+        fwd("up", X, u)
+        q.qlora_silu_gate_fwd(g, u, h)
+        fwd("down", h, y)
+        bwd("down", h, dY, dh, False)
+        q.qlora_silu_gate_bwd(dh, g, u, dg, du)
+        bwd("gate", X, dg, dx, False)
+        bwd("up", X, du, dx, True)
+    for _ in range(2):
+        mlp()
+    ms = graph_time(mlp, 3, flush)
+    fl = 2 * linear_flops(M, I, H, RANK_R, True) + linear_flops(M, H, I, RANK_R, True)
+    out["mlp_7b_fwd_bwd"] = {"us": ms * 1e3, "tflops": fl / ms / 1e9, "tokens_per_s": M / (ms * 1e-3),
+                             "frac_bf16_burst": fl / ms / 1e9 / peak, "flops": fl, "tokens": M}
+
+
 def components(dev, peaks) -> dict:
     """Quantize / dequantize (4096 x 4096 and 22016 x 8192, with outliers) and M = 16 forward of
     the 65B q_proj, each against the measured HBM copy bandwidth. Timed by
@@ -531,6 +666,13 @@ def components(dev, peaks) -> dict:
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for qn, qk, sfx in ((4096, 4096, ""), (22016, 8192, "_65b_gate")):
         _quant_components(q, synth, torch, dev, flush, peaks, out, qn, qk, sfx)
+    _seven_b_components(q, synth, torch, dev, flush, peaks, out)
+    # the NF4 expansion alone on every SM: the ceiling on the weight rate of any kernel that
+    # turns each weight into BF16 through the per-block table
+    per_clk, per_s = q.qlora_expand_rate(4096)
+    out["expansion_ceiling"] = {"weights_per_sm_clock": per_clk, "gweights_per_s": per_s / 1e9,
+                                "note": "nf4_build_lut + nf4_lookup8 per 64-block, codes from shared memory, "
+                                        "one CTA of 512 threads per SM, nothing else running"}
     # weight-stream bound forward at M = 16 (65B q_proj)
     n, k = 8192, 8192
     W = synth.weight(n, k).to(dev)
@@ -548,7 +690,9 @@ def components(dev, peaks) -> dict:
     ms = graph_time(fn, 50, flush)
     algo = n * k * (0.5 + 1.0 / 64 + 4.0 / 16384) + 2.0 * M_SMALL * (k + n) + 2.0 * RANK_R * (k + n)
     out["fwd_m16_q_proj"] = {"us": ms * 1e3, "gbs": algo / ms / 1e6, "frac": algo / ms / 1e6 / peaks["hbm_gbs"],
-                             "algo_bytes": algo}
+                             "algo_bytes": algo,
+                             "expansion_frac": n * k / (ms * 1e-3) / per_s,
+                             "expansion_bound_us": n * k / per_s * 1e6}
     # LoRA dropout (p = 0.05): q_proj forward + backward at 8192 tokens with and without it
     M = M_TOKENS
     X = synth.activations(M, k).to(dev)
@@ -806,7 +950,9 @@ def run_native(args) -> None:
             s = OracleSample()
             times = [s.step() for _ in range(args.cpu_steps)]
             v = s.flops * len(times) / sum(times) / 1e12
-            cpu = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": s.desc}
+            cpu = {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": s.desc,
+                   "extrapolated_step_ms": step_flops() / (v * 1e12) * 1e3,
+                   "configs": oracle_configs()}
     if world > 1:
         dist.barrier()
     if rank == 0:

@@ -37,6 +37,7 @@ EXPORTED = (
     "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
     "qlora_adamw_step", "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch",
+    "qlora_expand_rate",
 )
 
 
@@ -119,6 +120,7 @@ def lib() -> ctypes.CDLL:
         "qlora_timing_launch": (ctypes.c_int, [i32, vp, vp]),
         "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
         "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
+        "qlora_expand_rate": (ctypes.c_int, [i32, vp, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
         "qlora_linear_workspace_bytes_ex": (sz, [i64, i64, i64, i32, pd]),
         "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWConfig), vp]),
@@ -326,6 +328,14 @@ def qlora_silu_gate_bwd(dh, g, u, dg, du, stream=None):
 
 def qlora_selftest_wait_timeout(limit_ms: int = 100, stream=None) -> None:
     _check(lib().qlora_selftest_wait_timeout(int(limit_ms), _stream(stream)), "qlora_selftest_wait_timeout")
+
+
+def qlora_expand_rate(iters: int = 2048):
+    """(weights expanded per SM-clock, per second) of the NF4 table expansion alone."""
+    per_clk, per_s = ctypes.c_double(0), ctypes.c_double(0)
+    _check(lib().qlora_expand_rate(int(iters), ctypes.addressof(per_clk), ctypes.addressof(per_s)),
+           "qlora_expand_rate")
+    return per_clk.value, per_s.value
 
 
 def qlora_check_device_error(stream=None) -> None:

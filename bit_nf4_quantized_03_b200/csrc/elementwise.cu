@@ -304,6 +304,57 @@ cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
+// Expansion rate: how many weights per SM-clock the NF4 expansion itself sustains
+// when nothing else runs. Each thread repeatedly takes one 64-block's 32 bytes of
+// codes from shared memory, builds that block's table from a fresh scale and
+// looks up its 64 BF16 weights (nf4_build_lut + nf4_lookup8, the code the GEMM,
+// dequantize and merge kernels run); the results are folded so that none is
+// dead. Cycles are taken per CTA with clock64 around the loop.
+// ---------------------------------------------------------------------------
+constexpr int kExpandThreads = 512;
+__device__ unsigned long long g_expand_cycles[1024];
+__device__ uint32_t g_expand_sink;
+
+__global__ void __launch_bounds__(kExpandThreads, 1) expand_rate_kernel(const __grid_constant__ Nf4Table tab,
+                                                                        int iters) {
+  __shared__ __align__(16) uint32_t codes[kExpandThreads * 8];
+  for (int i = threadIdx.x; i < kExpandThreads * 8; i += blockDim.x)
+    codes[i] = 0x9E3779B9u * static_cast<uint32_t>(i + 1 + blockIdx.x * 977);
+  __syncthreads();
+  const uint4* mine = reinterpret_cast<const uint4*>(codes) + 2 * threadIdx.x;
+  float c = 0.01f + 1e-6f * static_cast<float>(threadIdx.x);
+  uint32_t acc = 0;
+  const unsigned long long t0 = clock64();
+  for (int it = 0; it < iters; ++it) {
+    const uint4 w0 = mine[0], w1 = mine[1];
+    const Nf4Lut lut = nf4_build_lut(tab, c);
+    c = __fadd_rn(c, 1e-7f);
+    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 o = nf4_lookup8(lut, ws[q] ^ static_cast<uint32_t>(it));
+      acc ^= o.x ^ o.y ^ o.z ^ o.w;
+    }
+  }
+  const unsigned long long t1 = clock64();
+  __syncthreads();
+  if (threadIdx.x == 0) g_expand_cycles[blockIdx.x] = t1 - t0;
+  if (acc == 0x5EEDF00Du) g_expand_sink = acc;
+}
+
+cudaError_t launch_expand_rate(const Nf4Table& tab, int iters, int grid, int* threads, cudaStream_t st) {
+  if (grid < 1 || grid > 1024 || iters < 1) return cudaErrorInvalidValue;
+  expand_rate_kernel<<<grid, kExpandThreads, 0, st>>>(tab, iters);
+  count_launches(1);
+  *threads = kExpandThreads;
+  return cudaGetLastError();
+}
+
+cudaError_t read_expand_cycles(unsigned long long* out, int grid) {
+  return cudaMemcpyFromSymbol(out, g_expand_cycles, sizeof(unsigned long long) * static_cast<size_t>(grid));
+}
+
+// ---------------------------------------------------------------------------
 // SiLU-gated glue: h = silu(g) * u ; dg = dh*u*sig*(1 + g*(1-sig)), du = dh*g*sig
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }

@@ -830,6 +830,34 @@ int qlora_selftest_wait_timeout(int32_t limit_ms, qlora_stream_t stream) {
                                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int qlora_expand_rate(int32_t iters, double* weights_per_sm_clock, double* weights_per_second) {
+  if (iters < 1 || iters > (1 << 20) || weights_per_sm_clock == nullptr || weights_per_second == nullptr)
+    return QLORA_ERR_INVALID;
+  const int grid = std::min(num_sms(), 1024);
+  cudaStream_t st = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return QLORA_ERR_CUDA;
+  int threads = 0;
+  int rc = QLORA_OK;
+  if (cudaEventRecord(e0, st) != cudaSuccess || launch_expand_rate(table(), iters, grid, &threads, st) != cudaSuccess ||
+      cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess)
+    rc = QLORA_ERR_CUDA;
+  float ms = 0.f;
+  std::vector<unsigned long long> cyc(static_cast<size_t>(grid), 0ull);
+  if (rc == QLORA_OK &&
+      (cudaEventElapsedTime(&ms, e0, e1) != cudaSuccess || read_expand_cycles(cyc.data(), grid) != cudaSuccess))
+    rc = QLORA_ERR_CUDA;
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (rc != QLORA_OK) return rc;
+  unsigned long long most = 1;
+  for (unsigned long long c : cyc) most = std::max(most, c);
+  const double per_cta = static_cast<double>(threads) * iters * 64.0;
+  *weights_per_sm_clock = per_cta / static_cast<double>(most);
+  *weights_per_second = per_cta * grid / (static_cast<double>(ms) * 1e-3);
+  return QLORA_OK;
+}
+
 int qlora_check_device_error(qlora_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;

@@ -179,6 +179,10 @@ cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, uint16_t*
                          float beta1, float beta2, float eps, float weight_decay, float grad_scale, int32_t step,
                          int num_sms, cudaStream_t st);
 cudaError_t launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t st);
+// Expansion-rate measurement (elementwise.cu): `grid` CTAs of *threads threads each
+// expand iters 64-blocks per thread; read_expand_cycles copies the per-CTA cycles.
+cudaError_t launch_expand_rate(const Nf4Table& tab, int iters, int grid, int* threads, cudaStream_t st);
+cudaError_t read_expand_cycles(unsigned long long* out, int grid);
 cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
                                  cudaStream_t st);
 cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,

@@ -338,6 +338,18 @@ int qlora_timing_launch(int32_t index, double *ms, double *flops);
  * QLORA_ERR_DEVICE once and the context stays usable. */
 int qlora_selftest_wait_timeout(int32_t limit_ms, qlora_stream_t stream);
 
+/* Measures how fast this library's NF4 expansion runs with nothing else on the
+ * SMs: one CTA per SM, each thread repeatedly building a 64-block's table
+ * bf16(fp32(L[j] * c)) and looking up its 64 BF16 weights from codes in
+ * shared memory, `iters` blocks per thread (1..2^20). Writes the weights
+ * expanded per SM-clock (the per-CTA clock64 count of the slowest CTA) and per
+ * second (CUDA events around the launch). This is the ceiling on the weight
+ * rate of any kernel that turns every weight into BF16 by this table, which
+ * bounds the few-token forward when memory does not. Runs on the legacy
+ * default stream of the current device and synchronizes it. The pages have no
+ * counterpart; it is a measuring tool. */
+int qlora_expand_rate(int32_t iters, double* weights_per_sm_clock, double* weights_per_second);
+
 /* Reads and clears the device error word (set when a kernel gave up on a
  * bounded wait). Synchronizes `stream`. Returns QLORA_OK or QLORA_ERR_DEVICE. */
 int qlora_check_device_error(qlora_stream_t stream);
