@@ -805,6 +805,25 @@ def run_case(args) -> None:
                 q.qlora_linear_bwd(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, ws)
             else:
                 q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+    elif name == "q_proj_7b":
+        # 7B q_proj fwd+bwd at 2048 tokens (4096 x 4096, r = 64)
+        M, N, K = 2048, 4096, 4096
+        W = synth.weight(N, K, layer=40).to(dev)
+        qw = q.QuantizedWeight(N, K, q.QLORA_SCALE_DQ_FP8, device=dev)
+        q.qlora_nf4_quantize(W, qw)
+        del W
+        a, b = (t.to(dev) for t in synth.lora_pair(RANK_R, K, N, layer=40))
+        x = synth.activations(M, K, layer=40).to(dev)
+        dy = synth.grad_output(M, N, layer=40).to(dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        u = torch.empty(M, RANK_R, dtype=torch.float32, device=dev)
+        da = torch.empty(RANK_R, K, dtype=torch.float32, device=dev)
+        db = torch.empty(N, RANK_R, dtype=torch.float32, device=dev)
+        ws = torch.empty(q.qlora_linear_workspace_bytes(M, N, K, RANK_R), dtype=torch.uint8, device=dev)
+        for _ in range(1 + args.case_iters):
+            q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+            q.qlora_linear_bwd(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, ws)
     elif name == "dropout_q_65b":
         n, k = LAYERS[0][1], LAYERS[0][2]
         m = M_TOKENS

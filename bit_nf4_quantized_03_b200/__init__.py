@@ -15,7 +15,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqlora.so")
+# QLORA_BOUNDS_CHECK=1 selects the bounds-checking build (python -m bit_nf4_quantized_03_b200.build --bounds-check)
+BOUNDS_CHECK = os.environ.get("QLORA_BOUNDS_CHECK", "") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libqlora_bounds.so" if BOUNDS_CHECK else "libqlora.so")
 
 QLORA_OK = 0
 QLORA_SCALE_BF16 = 0
@@ -37,7 +39,7 @@ EXPORTED = (
     "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
     "qlora_adamw_step", "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch",
-    "qlora_expand_rate",
+    "qlora_expand_rate", "qlora_bounds_site",
 )
 
 
@@ -121,6 +123,7 @@ def lib() -> ctypes.CDLL:
         "qlora_nf4_quantize_noalloc": (ctypes.c_int, [vp, pw, vp]),
         "qlora_selftest_wait_timeout": (ctypes.c_int, [i32, vp]),
         "qlora_expand_rate": (ctypes.c_int, [i32, vp, vp]),
+        "qlora_bounds_site": (ctypes.c_int, []),
         "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
         "qlora_linear_workspace_bytes_ex": (sz, [i64, i64, i64, i32, pd]),
         "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWConfig), vp]),
@@ -338,8 +341,16 @@ def qlora_expand_rate(iters: int = 2048):
     return per_clk.value, per_s.value
 
 
+def qlora_bounds_site() -> int:
+    """Site of the first failed bounds check since the last call (0: none); bounds-check build only."""
+    return int(lib().qlora_bounds_site())
+
+
 def qlora_check_device_error(stream=None) -> None:
-    _check(lib().qlora_check_device_error(_stream(stream)), "qlora_check_device_error")
+    rc = lib().qlora_check_device_error(_stream(stream))
+    if rc != QLORA_OK and BOUNDS_CHECK:
+        raise QloraError(rc, f"qlora_check_device_error (first failed bounds check: site {qlora_bounds_site()})")
+    _check(rc, "qlora_check_device_error")
 
 
 def qlora_launch_count() -> int:

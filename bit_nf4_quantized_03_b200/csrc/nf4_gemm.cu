@@ -287,31 +287,41 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           if (i < nmain) {
             const int kt = kt0 + i;
             mbar_arrive_expect_tx(bar, C::kABytes + C::kBBytes);
+            const int64_t kext = static_cast<int64_t>(p.k_tiles) * 64;    // reduction length, rounded up
             if (C::AMn) {
-              tma_load_2d(a_dst, &maps.a, bar, mb * 128, kt * 64);
-              tma_load_2d(a_dst + 8192, &maps.a, bar, mb * 128 + 64, kt * 64);
-            } else {
+              if (tma_start_ok(mb * 128, kt * 64, 2, p.rows, a_dst, 30))
+                tma_load_2d(a_dst, &maps.a, bar, mb * 128, kt * 64);
+              if (tma_start_ok(mb * 128 + 64, kt * 64, 2, p.rows + 64, a_dst + 8192, 31))
+                tma_load_2d(a_dst + 8192, &maps.a, bar, mb * 128 + 64, kt * 64);
+            } else if (tma_start_ok(kt * 64, mb * 128, 2, kext, a_dst, 32)) {
               tma_load_2d(a_dst, &maps.a, bar, kt * 64, mb * 128);
             }
             if (C::BMode == kB_TmaK) {
-              tma_load_2d(b_dst, &maps.b, bar, kt * 64, nb * C::BN);
+              if (tma_start_ok(kt * 64, nb * C::BN, 2, kext, b_dst, 33))
+                tma_load_2d(b_dst, &maps.b, bar, kt * 64, nb * C::BN);
             } else {
 #pragma unroll
               for (int j = 0; j < C::BN / 64; ++j) {
-                tma_load_2d(b_dst + j * 8192, &maps.b, bar, nb * C::BN + 64 * j, kt * 64);
-                if (C::HiLo) tma_load_2d(b_dst + C::kBTile + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, kt * 64);
+                if (tma_start_ok(nb * C::BN + 64 * j, kt * 64, 2, p.cols + 64 * j, b_dst + j * 8192, 34))
+                  tma_load_2d(b_dst + j * 8192, &maps.b, bar, nb * C::BN + 64 * j, kt * 64);
+                if (C::HiLo &&
+                    tma_start_ok(nb * C::BN + 64 * j, kt * 64, 2, p.cols + 64 * j, b_dst + C::kBTile + j * 8192, 35))
+                  tma_load_2d(b_dst + C::kBTile + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, kt * 64);
               }
             }
           } else {
             const int e = i - nmain;
             mbar_arrive_expect_tx(bar, C::kABytes + C::kBTile);
-            tma_load_2d(a_dst, &maps.a2, bar, e * 64, mb * 128);
+            if (tma_start_ok(e * 64, mb * 128, 2, p.ext_tiles * 64, a_dst, 36))
+              tma_load_2d(a_dst, &maps.a2, bar, e * 64, mb * 128);
             if (!C::BMn) {
-              tma_load_2d(b_dst, &maps.b2, bar, e * 64, nb * C::BN);
+              if (tma_start_ok(e * 64, nb * C::BN, 2, p.ext_tiles * 64, b_dst, 37))
+                tma_load_2d(b_dst, &maps.b2, bar, e * 64, nb * C::BN);
             } else {
 #pragma unroll
               for (int j = 0; j < C::BN / 64; ++j)
-                tma_load_2d(b_dst + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, e * 64);
+                if (tma_start_ok(nb * C::BN + 64 * j, e * 64, 2, p.cols + 64 * j, b_dst + j * 8192, 38))
+                  tma_load_2d(b_dst + j * 8192, &maps.b2, bar, nb * C::BN + 64 * j, e * 64);
             }
           }
           pending |= (1u << stage);

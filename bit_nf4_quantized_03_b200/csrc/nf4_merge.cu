@@ -175,7 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&code_empty[cs], cph ^ 1)) { ok = false; break; }
         cpend &= ~(1u << cs);
         mbar_arrive_expect_tx(&code_full[cs], kCodeTile);
-        tma_load_2d(sC + cs * kCodeTile, &map_codes, &code_full[cs], nb * (kMergeBN / 2), mb * 128);
+        if (tma_start_ok(nb * (kMergeBN / 2), mb * 128, 1, p.k / 2, sC + cs * kCodeTile, 40))
+          tma_load_2d(sC + cs * kCodeTile, &map_codes, &code_full[cs], nb * (kMergeBN / 2), mb * 128);
         cpend |= (1u << cs);
         cpar = (cpar & ~(1u << cs)) | (cph << cs);
         if (++cs == kCodeStages) { cs = 0; cph ^= 1; }
@@ -184,10 +185,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           opend &= ~(1u << os);
           uint64_t* bar = &op_full[os];
           mbar_arrive_expect_tx(bar, kATile + kBTile);
-          tma_load_2d(sA + os * kATile, &map_b, bar, ks * 64, mb * 128);
+          if (tma_start_ok(ks * 64, mb * 128, 2, p.k_steps * 64, sA + os * kATile, 41))
+            tma_load_2d(sA + os * kATile, &map_b, bar, ks * 64, mb * 128);
 #pragma unroll
           for (int j = 0; j < kMergeBN / 64; ++j)
-            tma_load_2d(sB + os * kBTile + j * 8192, &map_a, bar, nb * kMergeBN + 64 * j, ks * 64);
+            if (tma_start_ok(nb * kMergeBN + 64 * j, ks * 64, 2, p.k + 64 * j + 64, sB + os * kBTile + j * 8192, 42))
+              tma_load_2d(sB + os * kBTile + j * 8192, &map_a, bar, nb * kMergeBN + 64 * j, ks * 64);
           opend |= (1u << os);
           opar = (opar & ~(1u << os)) | (oph << os);
           if (++os == kOpStages) { os = 0; oph ^= 1; }
@@ -301,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           const int col = col0 + 32 * c;
           if (lane == 0) {
-            if (row0 < p.n && col < p.k) tma_store_2d(&map_out, sOut + ew * 2 * S::kChunk + sb * S::kChunk, col, row0);
+            if (row0 < p.n && col < p.k &&
+                tma_start_ok(col, row0, kF32 ? 4 : 2, p.k, sOut + ew * 2 * S::kChunk + sb * S::kChunk, 43))
+              tma_store_2d(&map_out, sOut + ew * 2 * S::kChunk + sb * S::kChunk, col, row0);
             bulk_commit_group();
           }
           ++issued;

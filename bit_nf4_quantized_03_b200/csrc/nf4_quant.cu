@@ -12,11 +12,14 @@
 #include <cstring>
 
 #include "qlora_device.cuh"
+#include <utility>
+
 #include "qlora_kernels.h"
 
 namespace qlora {
 
 __device__ int g_device_error = 0;
+__device__ int g_bounds_site = 0;
 
 // ---------------------------------------------------------------------------
 // Stage 1: absmax, codes, plain scales / fp32 absmax for double quant.
@@ -168,6 +171,10 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
     if (nfull > 0) tma_prefetch_desc(&wmap);
   }
   __syncthreads();
+  // launched with programmatic dependence: W may still be being written by the kernel
+  // before this one until this returns; the kernel after this one may be scheduled now
+  griddep_wait();
+  griddep_launch_dependents();
   auto issue = [&](int64_t i) {
     const int64_t b0 = (blockIdx.x + i * gridDim.x) * kQChunk;
     const int st = static_cast<int>(i % kQStages);
@@ -175,8 +182,10 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
       // rows past nfull arrive zero-filled and are counted in full
       uint8_t* dst = q_stage + st * kQStage;
       mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(kQStage));
-      tma_load_2d(dst, &wmap, &full[st], 0, static_cast<int32_t>(b0));
-      tma_load_2d(dst + kQStage / 2, &wmap, &full[st], 32, static_cast<int32_t>(b0));
+      if (tma_start_ok(0, static_cast<int32_t>(b0), 4, 64, dst, 50) && qlora_check(b0 < nfull, 51))
+        tma_load_2d(dst, &wmap, &full[st], 0, static_cast<int32_t>(b0));
+      if (tma_start_ok(32, static_cast<int32_t>(b0), 4, 64, dst + kQStage / 2, 52))
+        tma_load_2d(dst + kQStage / 2, &wmap, &full[st], 32, static_cast<int32_t>(b0));
     } else {
       mbar_arrive(&full[st]);                  // only the ragged last block: read from global memory
     }
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
       word.w = nf4_codes8(v[6], v[7], inv, s_tab);
     }
     if (cls == 0) {
-      *reinterpret_cast<uint4*>(codes + b * 32 + h * 16) = word;
+      if (qlora_check((b + 1) * 64 <= n_elem, 53)) *reinterpret_cast<uint4*>(codes + b * 32 + h * 16) = word;
     } else if (cls == 1) {
       // only the bytes that hold present elements; an odd tail keeps its high nibble 0
       const uint32_t ww[4] = {word.x, word.y, word.z, word.w};
@@ -271,6 +280,8 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
 __global__ void __launch_bounds__(1024) dq_mean_kernel(const double* __restrict__ part, int64_t nchunks,
                                                        int64_t nblk, float* __restrict__ mean_out) {
   __shared__ double tree_buf[2 * kTreeBuf];
+  griddep_wait();                      // the partials of stage 1 are complete and visible
+  griddep_launch_dependents();
   const double S = tree_sum_cta(part, nchunks, tree_buf);
   if (threadIdx.x == 0) *mean_out = static_cast<float>(S / static_cast<double>(nblk));
 }
@@ -286,6 +297,8 @@ __global__ void __launch_bounds__(256) dq_finish_kernel(const float* __restrict_
                                                          const float* __restrict__ absmax, int64_t nblk,
                                                          uint8_t* __restrict__ q_out, float* __restrict__ s2_out) {
   __shared__ float wmax[kFinishPer][8];
+  griddep_wait();                      // the mean (and, before it, stage 1's absmax values) are visible
+  griddep_launch_dependents();
   const int64_t nb2 = (nblk + 255) / 256;
   float a[kFinishPer];
 #pragma unroll
@@ -342,7 +355,6 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
   const int64_t nfull = n_elem / 64;
   const int64_t nchunks = (nfull + kDChunk - 1) / kDChunk;
   const int64_t my_n = (nchunks > blockIdx.x) ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const float mean = (ss.dq_mean != nullptr) ? __ldg(ss.dq_mean) : 0.f;
   uint8_t* ring = d_smem;
   const uint32_t stage_out = smem_u32(d_smem + kDStages * kDChunk * 32 + warp * 4096);
   if (tid == 0) {
@@ -350,6 +362,10 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
     fence_mbar_init();
   }
   __syncthreads();
+  // launched with programmatic dependence: the codes and scales may still be being written
+  // by the kernel before this one until this returns
+  griddep_wait();
+  griddep_launch_dependents();
   auto issue = [&](int64_t i) {
     const int64_t b0 = (blockIdx.x + i * gridDim.x) * kDChunk;
     int64_t nb = nfull - b0;
@@ -360,6 +376,7 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
   };
   if (tid == 0)
     for (int64_t i = 0; i < my_n && i < kDStages; ++i) issue(i);
+  const float mean = (ss.dq_mean != nullptr) ? __ldg(ss.dq_mean) : 0.f;
   const uint32_t x = (lane >> 2) & 1;           // read order that keeps the two 16-byte loads conflict-free
   // the scale of this lane's block in the next chunk is loaded one chunk ahead
   float c_next = 0.f;
@@ -377,7 +394,7 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
       if (i + 1 < my_n && bn < nfull) c_next = block_scale(ss, bn, mean);
     }
     if (!mbar_wait(&full[st], static_cast<uint32_t>((i / kDStages) & 1))) break;
-    if (b < nfull) {
+    if (b < nfull && qlora_check(b0 >= 0, 54)) {
       const uint32_t src = smem_u32(ring + st * (kDChunk * 32) + (warp * 32 + lane) * 32);
       uint4 h0, h1;
       asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -406,7 +423,7 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
       const int o = it * 512 + lane * 16;     // byte offset in the warp's 4 KB of output
       const int blk = o >> 7;
       const int chunk = (o >> 4) & 7;
-      if (blk < nvalid) {
+      if (blk < nvalid && qlora_check((b0 + blk + 1) * 64 <= n_elem, 55)) {
         uint4 v;
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
@@ -435,6 +452,27 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
+
+// Launch with programmatic dependent launch allowed: the kernel may be scheduled while
+// the one before it on the stream finishes; each kernel here waits (griddepcontrol.wait)
+// before it reads anything that kernel may write.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, int smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(block), 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launches(1);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 template <typename K>
 static cudaError_t set_smem_once(K kernel, int bytes, bool* done) {
@@ -471,9 +509,8 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   if (!dq) {
     e = set_smem_once(nf4_quantize_kernel<false>, kQSmem, smem_set[0]);
     if (e != cudaSuccess) return e;
-    nf4_quantize_kernel<false><<<grid, 256, kQSmem, st>>>(wmap, W, n_elem, bk, codes, scale_bf16, nullptr, nullptr);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_pdl(nf4_quantize_kernel<false>, grid, 256, kQSmem, st, wmap, W, n_elem, bk, codes, scale_bf16,
+                      static_cast<float*>(nullptr), static_cast<double*>(nullptr));
   }
   const QuantWsLayout L = quant_ws_layout(n_elem);
   float* absmax = reinterpret_cast<float*>(static_cast<char*>(ws) + L.absmax_off);
@@ -481,23 +518,19 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   // stage 1 also writes one fp64 tree sum per chunk (the first levels of the fixed-order sum)
   e = set_smem_once(nf4_quantize_kernel<true>, kQSmem, smem_set[1]);
   if (e != cudaSuccess) return e;
-  nf4_quantize_kernel<true><<<grid, 256, kQSmem, st>>>(wmap, W, n_elem, bk, codes, nullptr, absmax, part_a);
-  count_launches(1);
-  e = cudaGetLastError();
+  e = launch_pdl(nf4_quantize_kernel<true>, grid, 256, kQSmem, st, wmap, W, n_elem, bk, codes,
+                 static_cast<uint16_t*>(nullptr), absmax, part_a);
   if (e != cudaSuccess) return e;
   // the rest of the tree and the mean (one CTA), then the E4M3 pass
-  dq_mean_kernel<<<1, 1024, 0, st>>>(part_a, nchunks, nblk, dq_mean);
-  count_launches(1);
-  e = cudaGetLastError();
+  e = launch_pdl(dq_mean_kernel, 1, 1024, 0, st, static_cast<const double*>(part_a), nchunks, nblk, dq_mean);
   if (e != cudaSuccess) return e;
   const int64_t nb2 = (nblk + 255) / 256;
   // enough CTAs that each takes at most kFinishPer 256-blocks, at least one per SM when there is work
   int64_t g2 = (nb2 + kFinishPer - 1) / kFinishPer;
   if (g2 < num_sms) g2 = nb2 < num_sms ? nb2 : num_sms;
   const int grid2 = static_cast<int>(g2);
-  dq_finish_kernel<<<grid2, 256, 0, st>>>(dq_mean, absmax, nblk, scale_fp8, dq_scale);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(dq_finish_kernel, grid2, 256, 0, st, static_cast<const float*>(dq_mean),
+                    static_cast<const float*>(absmax), nblk, scale_fp8, dq_scale);
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t n_elem, const Nf4Table& tab,
@@ -509,9 +542,7 @@ cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t 
   const int64_t nchunks = (nfull + kDChunk - 1) / kDChunk;
   int64_t grid = nchunks < 3LL * num_sms ? nchunks : 3LL * num_sms;
   if (grid < 1) grid = 1;
-  nf4_dequantize_kernel<<<static_cast<int>(grid), 256, kDSmem, st>>>(codes, ss, n_elem, tab, out);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(nf4_dequantize_kernel, static_cast<int>(grid), 256, kDSmem, st, codes, ss, n_elem, tab, out);
 }
 
 }  // namespace qlora

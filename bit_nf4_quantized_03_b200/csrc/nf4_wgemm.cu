@@ -111,6 +111,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 template <int kCount>
 __device__ __forceinline__ void wstore(const GemmParams& p, int split, int feat, int tok0, const uint32_t (&v)[32]) {
   if (feat >= p.rows) return;
+  if (!qlora_check(feat < p.ld_out && tok0 >= 0 && (p.out_mode != kOutPartial || split < p.splits), 17)) return;
   const int64_t ld = p.ld_out;
   const int nvalid = p.cols - tok0;     // tokens of the chunk inside the output (may be < kCount or <= 0)
   if (p.accumulate && p.out_mode != kOutPartial) {
@@ -229,23 +230,32 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           if (i < nmain) {
             const int kt = kt0 + i;
             mbar_arrive_expect_tx(bar, C::kRBytes + C::kBTile);
-            if (C::Bwd) tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, mb * 64, kt * 64);
-            else tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, kt * 32, mb * 128);
+            if (C::Bwd) {
+              if (tma_start_ok(mb * 64, kt * 64, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 10))
+                tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, mb * 64, kt * 64);
+            } else if (tma_start_ok(kt * 32, mb * 128, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 11)) {
+              tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, kt * 32, mb * 128);
+            }
 #pragma unroll
             for (int t = 0; t < C::NAcc; ++t)
-              tma_load_2d(b_dst + t * (C::BN * 128), &maps.act, bar, kt * 64, nb * C::TOK + t * C::BN);
+              if (tma_start_ok(kt * 64, nb * C::TOK + t * C::BN, 2, C::Bwd ? p.w_rows : p.w_kblocks * 64,
+                               b_dst + t * (C::BN * 128), 12))
+                tma_load_2d(b_dst + t * (C::BN * 128), &maps.act, bar, kt * 64, nb * C::TOK + t * C::BN);
           } else {
             const int e = i - nmain;
             mbar_arrive_expect_tx(bar, C::kATile + C::kBTile);
             if (C::Bwd) {
-              tma_load_2d(a_dst, &maps.a2, bar, mb * 128, e * 64);
-              tma_load_2d(a_dst + 8192, &maps.a2, bar, mb * 128 + 64, e * 64);
-            } else {
+              if (tma_start_ok(mb * 128, e * 64, 2, p.w_kblocks * 64, a_dst, 13))
+                tma_load_2d(a_dst, &maps.a2, bar, mb * 128, e * 64);
+              if (tma_start_ok(mb * 128 + 64, e * 64, 2, p.w_kblocks * 64, a_dst + 8192, 14))
+                tma_load_2d(a_dst + 8192, &maps.a2, bar, mb * 128 + 64, e * 64);
+            } else if (tma_start_ok(e * 64, mb * 128, 2, p.ext_tiles * 64, a_dst, 15)) {
               tma_load_2d(a_dst, &maps.a2, bar, e * 64, mb * 128);
             }
 #pragma unroll
             for (int t = 0; t < C::NAcc; ++t)
-              tma_load_2d(b_dst + t * (C::BN * 128), &maps.b2, bar, e * 64, nb * C::TOK + t * C::BN);
+              if (tma_start_ok(e * 64, nb * C::TOK + t * C::BN, 2, p.ext_tiles * 64, b_dst + t * (C::BN * 128), 16))
+                tma_load_2d(b_dst + t * (C::BN * 128), &maps.b2, bar, e * 64, nb * C::TOK + t * C::BN);
           }
           pending |= (1u << stage);
           pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
@@ -656,13 +666,19 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           if (i < nmain) {
             const int kt = kt0 + i;
             mbar_arrive_expect_tx(&codes_full[stage], C::kRBytes);
-            if (C::Bwd) tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], mh * 64, kt * 64);
-            else tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], kt * 32, mh * 128);
+            if (C::Bwd) {
+              if (tma_start_ok(mh * 64, kt * 64, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 20))
+                tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], mh * 64, kt * 64);
+            } else if (tma_start_ok(kt * 32, mh * 128, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 21)) {
+              tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], kt * 32, mh * 128);
+            }
             pend_codes |= (1u << stage);
             if (even) mbar_arrive_expect_tx(&tma_full[stage], 2 * C::kBStage);
 #pragma unroll
             for (int t = 0; t < C::NT; ++t)
-              tma_load_2d_pair(b_dst + t * C::kBTile, &maps.act, full_e, kt * 64, tok0 + t * C::BN);
+              if (tma_start_ok(kt * 64, tok0 + t * C::BN, 2, C::Bwd ? p.w_rows : p.w_kblocks * 64,
+                               b_dst + t * C::kBTile, 22))
+                tma_load_2d_pair(b_dst + t * C::kBTile, &maps.act, full_e, kt * 64, tok0 + t * C::BN);
           } else {
             const int e = i - nmain;
             // no codes for an extension step: complete codes_full's phase anyway, so that its
@@ -670,14 +686,17 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_arrive(&codes_full[stage]);
             if (even) mbar_arrive_expect_tx(&tma_full[stage], 2 * (C::kATile + C::kBStage));
             if (C::Bwd) {
-              tma_load_2d_pair(a_dst, &maps.a2, full_e, mh * 128, e * 64);
-              tma_load_2d_pair(a_dst + 8192, &maps.a2, full_e, mh * 128 + 64, e * 64);
-            } else {
+              if (tma_start_ok(mh * 128, e * 64, 2, p.w_kblocks * 64, a_dst, 23))
+                tma_load_2d_pair(a_dst, &maps.a2, full_e, mh * 128, e * 64);
+              if (tma_start_ok(mh * 128 + 64, e * 64, 2, p.w_kblocks * 64, a_dst + 8192, 24))
+                tma_load_2d_pair(a_dst + 8192, &maps.a2, full_e, mh * 128 + 64, e * 64);
+            } else if (tma_start_ok(e * 64, mh * 128, 2, p.ext_tiles * 64, a_dst, 25)) {
               tma_load_2d_pair(a_dst, &maps.a2, full_e, e * 64, mh * 128);
             }
 #pragma unroll
             for (int t = 0; t < C::NT; ++t)
-              tma_load_2d_pair(b_dst + t * C::kBTile, &maps.b2, full_e, e * 64, tok0 + t * C::BN);
+              if (tma_start_ok(e * 64, tok0 + t * C::BN, 2, p.ext_tiles * 64, b_dst + t * C::kBTile, 26))
+                tma_load_2d_pair(b_dst + t * C::kBTile, &maps.b2, full_e, e * 64, tok0 + t * C::BN);
           }
           pend_full |= (1u << stage);
           pend_par = (pend_par & ~(1u << stage)) | (ph << stage);

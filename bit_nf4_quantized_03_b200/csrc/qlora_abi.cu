@@ -134,6 +134,15 @@ int num_sms() {
 }
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+}  // namespace
+
+namespace qlora {
+const Nf4Table& host_table() { return table(); }
+const Nf4Buckets& host_buckets() { return buckets(); }
+int host_num_sms() { return num_sms(); }
+}  // namespace qlora
+
+namespace {
 
 bool weight_ok(const qlora_nf4_weight* w) {
   if (w == nullptr || w->n < 1 || w->k < 1) return false;
@@ -436,6 +445,7 @@ const char* qlora_status_string(int s) {
     case QLORA_ERR_CUDA: return "CUDA error";
     case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
     case QLORA_ERR_DEVICE: return "a kernel gave up on a bounded wait";
+    case QLORA_ERR_BOUNDS: return "a bounds check failed (bounds-checking build)";
     default: return "unknown status";
   }
 }
@@ -866,9 +876,19 @@ int qlora_check_device_error(qlora_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(qlora::g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
-    return QLORA_ERR_DEVICE;
+    return v == qlora::kErrBounds ? QLORA_ERR_BOUNDS : QLORA_ERR_DEVICE;
   }
   return QLORA_OK;
+}
+
+int qlora_bounds_site(void) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, qlora::g_bounds_site, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(qlora::g_bounds_site, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
 }
 
 }  // extern "C"

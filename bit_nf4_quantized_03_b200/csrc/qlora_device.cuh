@@ -31,8 +31,9 @@ struct Nf4Buckets {
 
 // Device error word: kernels write a non-zero code here when a bounded wait
 // gives up, so the host can read the failure instead of the GPU hanging.
-enum : int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadLayout = 2 };   // values of g_device_error
+enum : int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadLayout = 2, kErrBounds = 3 };   // values of g_device_error
 extern __device__ int g_device_error;
+extern __device__ int g_bounds_site;       // first failed bounds check (bounds-check build)
 
 // ---------------------------------------------------------------------------
 // small helpers
@@ -58,6 +59,50 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
+}
+
+// ---------------------------------------------------------------------------
+// Bounds checks. In a build with -DQLORA_BOUNDS_CHECK (build.py --bounds-check)
+// qlora_check records a failed condition -- kErrBounds in the error word and the
+// site number in g_bounds_site, first failure kept -- and returns false, so the
+// caller skips the access it guards (a skipped TMA load then leaves its barrier
+// incomplete, and the bounded waits end the kernel). No assert, no trap. In the
+// normal build both helpers are constant true and cost nothing.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool qlora_check(bool ok, int site) {
+#ifdef QLORA_BOUNDS_CHECK
+  if (!ok) {
+    atomicCAS(&g_bounds_site, 0, site);
+    atomicExch(&g_device_error, kErrBounds);
+  }
+  return ok;
+#else
+  (void)ok;
+  (void)site;
+  return true;
+#endif
+}
+
+// Start of a 2D TMA tile: x (innermost, in elements of elem_bytes) on a 16-byte
+// boundary, x and y not negative, shared-memory address 16-byte aligned, and x
+// less than one tile (256 elements) past the tensor's inner extent. A tile may
+// start past the edge by design on ragged shapes -- the load reads the fill
+// value there -- but a start further out means a wrong plan.
+__device__ __forceinline__ bool tma_start_ok(int32_t x, int32_t y, int elem_bytes, int64_t inner, const void* smem,
+                                             int site) {
+#ifdef QLORA_BOUNDS_CHECK
+  return qlora_check(x >= 0 && y >= 0 && (static_cast<int64_t>(x) * elem_bytes) % 16 == 0 && x < inner + 256 &&
+                         (static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 15u) == 0,
+                     site);
+#else
+  (void)x;
+  (void)y;
+  (void)elem_bytes;
+  (void)inner;
+  (void)smem;
+  (void)site;
+  return true;
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -112,7 +157,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar_ptr, uint32_t parity) {
   while (true) {
     if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
     if ((++tries & 15u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicExch(&g_device_error, kErrWaitTimeout);
+      atomicCAS(&g_device_error, kErrNone, kErrWaitTimeout);   // an earlier error (its cause) is kept
       return false;
     }
   }
@@ -156,6 +201,10 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 // Contiguous bulk copy global -> shared (TMA engine, no tensor map, no
 // multicast). Addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  if (!qlora_check(bytes > 0 && (bytes & 15u) == 0 && (reinterpret_cast<uintptr_t>(gsrc) & 15u) == 0 &&
+                       (static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst)) & 15u) == 0,
+                   90))
+    return;
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(smem_dst)),
                "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))

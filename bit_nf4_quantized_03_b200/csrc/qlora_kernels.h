@@ -38,6 +38,11 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
                             float* dq_mean, void* ws, int num_sms, cudaStream_t st);
 // Bucket table of the quantizer's code search, built from the 15 midpoints (qlora_abi.cu).
 Nf4Buckets nf4_buckets_from_midpoints(const float* mid);
+// The level table and bucket table every entry point uses, and the SM count of the
+// current device (qlora_abi.cu; built once, cached).
+const Nf4Table& host_table();
+const Nf4Buckets& host_buckets();
+int host_num_sms();
 cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t n_elem, const Nf4Table& tab,
                               uint16_t* out, int num_sms, cudaStream_t st);
 

@@ -72,7 +72,8 @@ typedef enum {
   QLORA_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels cover */
   QLORA_ERR_CUDA = 3,        /* a CUDA launch or query failed */
   QLORA_ERR_WORKSPACE = 4,   /* workspace pointer null or too small */
-  QLORA_ERR_DEVICE = 5       /* a kernel gave up on a bounded wait */
+  QLORA_ERR_DEVICE = 5,      /* a kernel gave up on a bounded wait */
+  QLORA_ERR_BOUNDS = 6       /* a bounds check failed (bounds-checking build only) */
 } qlora_status;
 
 typedef enum {
@@ -149,6 +150,9 @@ int qlora_nf4_quantize(const float *W, qlora_nf4_weight *w, void *ws, size_t ws_
  *    larger requests return QLORA_ERR_UNSUPPORTED with nothing enqueued.
  *  - The first call on a device looks up the scratch's device address with
  *    that device current; make that first call before any stream capture.
+ *    The address is kept per device and context: the first call after the
+ *    device's context was destroyed and created again (cudaDeviceReset)
+ *    looks it up again, so that call, too, belongs before any capture.
  *  - All calls share the one array, which keeps the last call's contents
  *    (each call writes every scratch word before reading it). Calls whose
  *    work overlaps on the GPU -- on different streams, or from different host
@@ -351,8 +355,19 @@ int qlora_selftest_wait_timeout(int32_t limit_ms, qlora_stream_t stream);
 int qlora_expand_rate(int32_t iters, double* weights_per_sm_clock, double* weights_per_second);
 
 /* Reads and clears the device error word (set when a kernel gave up on a
- * bounded wait). Synchronizes `stream`. Returns QLORA_OK or QLORA_ERR_DEVICE. */
+ * bounded wait, or, in the bounds-checking build, when a check failed).
+ * Synchronizes `stream`. Returns QLORA_OK, QLORA_ERR_DEVICE or QLORA_ERR_BOUNDS. */
 int qlora_check_device_error(qlora_stream_t stream);
+
+/* Bounds-checking build (compiled with -DQLORA_BOUNDS_CHECK): the kernels check
+ * each TMA tile start (innermost coordinate on a 16-byte boundary and inside
+ * the tensor, shared-memory address aligned), each bulk copy (16-byte aligned
+ * addresses and size) and the main global stores against the sizes the host
+ * planned; a failed check skips the access and records QLORA_ERR_BOUNDS and
+ * the site number. This returns the first failing site since the last call
+ * and clears it (0: none; always 0 in the normal build; -1: CUDA error). It
+ * stands in for an external memory checker where none can run. */
+int qlora_bounds_site(void);
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ MAX_ABS_RMS = 1e-2     # max |error| / RMS(reference)
 
 def ensure_built():
     from bit_nf4_quantized_03_b200 import build
-    build.build()
+    build.build(bounds_check=q.BOUNDS_CHECK)
     q.lib()
 
 

@@ -36,6 +36,16 @@ def test_library_exports_every_declared_symbol(L):
     assert sorted(q.EXPORTED) == syms
 
 
+def test_bounds_checking_build_exports_the_same_symbols():
+    # the -DQLORA_BOUNDS_CHECK variant is the same ABI (built by the build step next to libqlora.so)
+    from bit_nf4_quantized_03_b200 import build
+    if not os.path.exists(build.LIB_BOUNDS):
+        pytest.skip("bounds-checking build not present (python -m bit_nf4_quantized_03_b200.build --bounds-check)")
+    LB = ctypes.CDLL(build.LIB_BOUNDS)
+    for s in _declared_symbols():
+        assert hasattr(LB, s), s
+
+
 def test_timing_launch_rejects_indexes_without_a_record(L):
     # host bookkeeping only: before any timed launch there is no record to read (1 = QLORA_ERR_INVALID)
     ms, fl = ctypes.c_double(0), ctypes.c_double(0)

@@ -6,7 +6,12 @@ device memory), or a latency-critical path that must not call cudaMalloc.
 qlora_nf4_quantize_noalloc serves them from a fixed scratch array inside the
 library. These tests call it through the C ABI and require the same bytes as
 qlora_nf4_quantize, on two calls in a row (the second call reuses the scratch
-the first one left behind). This file is collected last on purpose.
+the first one left behind).
+
+The file name sorts last, so pytest collects it after every other test file: a
+run that stops at the first failure (-x) has then already run the rest of the
+suite when one of these fails. The tests themselves depend on no order; they
+pass alone in a fresh process as well.
 """
 import ctypes
 
