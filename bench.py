@@ -47,9 +47,9 @@ L2_FLUSH_BYTES = 512 << 20
 PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12) flops, one at 16 tokens <= 5.8e9
 
 # DRAM bytes (read + write) per launch of the CTA-pair fused GEMM, averaged over its 14 launches of one step, from the
-# 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum; summary in
-# profiles/launch_list_65b_decoder_step.md). Printed only while the kernel's sources hash to the value
-# recorded with it; any change to them prints null until the counters are taken again.
+# 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum). Printed only while the
+# kernel's sources hash to the value recorded with it; any change to them prints null until the counters are taken
+# again.
 WGEMM_TRAFFIC = {"bytes_per_launch": 920445495,
                  "sources_sha256": "3959e96c205beb70922c1f9ff599d89536741d9f65ddc973e784c89b05be6ea5"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
