@@ -57,6 +57,7 @@ __device__ __forceinline__ uint4 apply_bits(uint4 x, uint32_t bits) {
 __global__ void __launch_bounds__(256) dropout_mask_kernel(const uint4* __restrict__ X, int64_t groups, uint32_t thr,
                                                            uint64_t seed, uint64_t offset, uint4* __restrict__ Xd,
                                                            uint8_t* __restrict__ mask) {
+  griddep_enter();
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   const uint32_t c2 = static_cast<uint32_t>(offset), c3 = static_cast<uint32_t>(offset >> 32);
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(256) dropout_mask_kernel(const uint4* __restri
 
 __global__ void __launch_bounds__(256) mask_apply_kernel(const uint4* __restrict__ X, int64_t groups,
                                                          const uint8_t* __restrict__ mask, uint4* __restrict__ Xd) {
+  griddep_enter();
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
        g += static_cast<int64_t>(gridDim.x) * blockDim.x)
     Xd[g] = apply_bits(__ldcs(X + g), __ldg(mask + g));
@@ -92,18 +94,14 @@ int grid_for(int64_t groups) {
 cudaError_t launch_dropout_mask(const uint16_t* X, int64_t count, uint32_t thr, uint64_t seed, uint64_t offset,
                                 uint16_t* Xd, uint8_t* mask, cudaStream_t st) {
   const int64_t groups = count / 8;
-  dropout_mask_kernel<<<grid_for(groups), 256, 0, st>>>(reinterpret_cast<const uint4*>(X), groups, thr, seed, offset,
-                                                        reinterpret_cast<uint4*>(Xd), mask);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(dropout_mask_kernel, grid_for(groups), 256, 0, st, 1, reinterpret_cast<const uint4*>(X), groups,
+                    thr, seed, offset, reinterpret_cast<uint4*>(Xd), mask);
 }
 
 cudaError_t launch_mask_apply(const uint16_t* X, int64_t count, const uint8_t* mask, uint16_t* Xd, cudaStream_t st) {
   const int64_t groups = count / 8;
-  mask_apply_kernel<<<grid_for(groups), 256, 0, st>>>(reinterpret_cast<const uint4*>(X), groups, mask,
-                                                      reinterpret_cast<uint4*>(Xd));
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(mask_apply_kernel, grid_for(groups), 256, 0, st, 1, reinterpret_cast<const uint4*>(X), groups,
+                    mask, reinterpret_cast<uint4*>(Xd));
 }
 
 }  // namespace qlora

@@ -9,6 +9,21 @@ namespace qlora {
 __device__ __forceinline__ uint16_t f2bf(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
+// sum over t < splits of src[t * stride], in the order t = 0, 1, ... (the same value as a
+// plain loop), with eight loads in flight at a time instead of one
+__device__ __forceinline__ float sum_splits(const float* __restrict__ src, int splits, int64_t stride) {
+  float s = 0.f;
+  for (int t0 = 0; t0 < splits; t0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = (t0 + u < splits) ? __ldcg(src + static_cast<int64_t>(t0 + u) * stride) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t0 + u < splits) s += v[u];
+  }
+  return s;
+}
+
 static int blocks_for(int64_t n, int threads) {
   int64_t g = (n + threads - 1) / threads;
   if (g > 148 * 32) g = 148 * 32;
@@ -17,18 +32,20 @@ static int blocks_for(int64_t n, int threads) {
 
 // U (or G) = sum over split partials [split][rows][r_pad], fixed order.
 // Writes any of: fp32 [rows, r]; bf16(scale * U) [rows, r_pad]; hi/lo bf16 [rows, r_pad].
+// With `extra_src`, the same pass also splits a second fp32 [rows, r] matrix into hi/lo
+// bf16 [rows, r_pad] (the saved U next to G in the backward): one launch for both.
 __global__ void lora_finalize_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
                                      int r, int r_pad, float scale, float* __restrict__ out_f32,
                                      uint16_t* __restrict__ out_scaled, uint16_t* __restrict__ out_hi,
-                                     uint16_t* __restrict__ out_lo, float pre) {
+                                     uint16_t* __restrict__ out_lo, float pre, const float* __restrict__ extra_src,
+                                     uint16_t* __restrict__ extra_hi, uint16_t* __restrict__ extra_lo) {
+  griddep_enter();
   const int64_t total = rows * r_pad;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t row = idx / r_pad;
     const int j = static_cast<int>(idx - row * r_pad);
-    float s = 0.f;
-    if (j < r)
-      for (int t = 0; t < splits; ++t) s += part[t * part_stride + idx];
+    float s = (j < r) ? sum_splits(part + idx, splits, part_stride) : 0.f;
     s = __fmul_rn(pre, s);
     if (out_f32 != nullptr && j < r) out_f32[row * r + j] = s;
     if (out_scaled != nullptr) out_scaled[idx] = f2bf(__fmul_rn(scale, s));
@@ -37,76 +54,95 @@ __global__ void lora_finalize_kernel(const float* __restrict__ part, int splits,
       out_hi[idx] = h;
       out_lo[idx] = f2bf(__fsub_rn(s, bf2f(h)));
     }
+    if (extra_src != nullptr) {
+      const float e = (j < r) ? extra_src[row * r + j] : 0.f;
+      const uint16_t h = f2bf(e);
+      extra_hi[idx] = h;
+      extra_lo[idx] = f2bf(__fsub_rn(e, bf2f(h)));
+    }
   }
 }
 
 cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows, int32_t r,
                                  int32_t r_pad, float scale, float* out_f32, uint16_t* out_scaled_bf16,
-                                 uint16_t* out_hi, uint16_t* out_lo, cudaStream_t st, float pre) {
+                                 uint16_t* out_hi, uint16_t* out_lo, cudaStream_t st, float pre,
+                                 const float* extra_src, uint16_t* extra_hi, uint16_t* extra_lo) {
   const int64_t total = rows * r_pad;
-  lora_finalize_kernel<<<blocks_for(total, 256), 256, 0, st>>>(part, splits, part_stride, rows, r, r_pad, scale,
-                                                                out_f32, out_scaled_bf16, out_hi, out_lo, pre);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(lora_finalize_kernel, blocks_for(total, 256), 256, 0, st, 1, part, splits, part_stride, rows,
+                    static_cast<int>(r), static_cast<int>(r_pad), scale, out_f32, out_scaled_bf16, out_hi, out_lo,
+                    pre, extra_src, extra_hi, extra_lo);
 }
 
-__global__ void split_hilo_kernel(const float* __restrict__ src, int64_t rows, int r, int r_pad,
-                                  uint16_t* __restrict__ hi, uint16_t* __restrict__ lo) {
-  const int64_t total = rows * r_pad;
-  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = idx / r_pad;
-    const int j = static_cast<int>(idx - row * r_pad);
-    const float s = (j < r) ? src[row * r + j] : 0.f;
-    const uint16_t h = f2bf(s);
-    hi[idx] = h;
-    lo[idx] = f2bf(__fsub_rn(s, bf2f(h)));
-  }
-}
-
-cudaError_t launch_split_hilo(const float* src, int64_t rows, int32_t r, int32_t r_pad, uint16_t* hi, uint16_t* lo,
-                              cudaStream_t st) {
-  split_hilo_kernel<<<blocks_for(rows * r_pad, 256), 256, 0, st>>>(src, rows, r, r_pad, hi, lo);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
-// dB[row, j] (or dA[j, row] when transposed) (+)= scale * sum_t part[t][row][j]
+// dB[row, j] (+)= scale * sum_t part[t][row][j]
 __global__ void grad_finalize_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
-                                     int r, int ld_part, float scale, float* __restrict__ out, int transpose,
-                                     int accumulate) {
+                                     int r, int ld_part, float scale, float* __restrict__ out, int accumulate) {
+  griddep_enter();
   const int64_t total = rows * r;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    int64_t row, j;
-    if (transpose) {   // consecutive threads walk the contiguous dimension of dA [r, rows]
-      j = idx / rows;
-      row = idx - j * rows;
-    } else {
-      row = idx / r;
-      j = idx - row * r;
+    const int64_t row = idx / r;
+    const int64_t j = idx - row * r;
+    const float s = __fmul_rn(scale, sum_splits(part + row * ld_part + j, splits, part_stride));
+    out[idx] = accumulate ? (out[idx] + s) : s;
+  }
+}
+
+// dA[j, row] (+)= scale * sum_t part[t][row][j]: 32 x 32 tiles through shared memory, so
+// that both the partials (rows of ld_part) and dA (rows of `rows`) are read and written
+// along their contiguous dimension. 256 threads: warp w sums rows w, w + 8, ... of the
+// tile (lane = j), then writes j = w, w + 8, ... (lane = row).
+__global__ void __launch_bounds__(256) grad_finalize_t_kernel(const float* __restrict__ part, int splits,
+                                                              int64_t part_stride, int64_t rows, int r, int ld_part,
+                                                              float scale, float* __restrict__ out, int accumulate) {
+  griddep_enter();
+  __shared__ float tile[32][33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tr = (rows + 31) / 32;
+  const int64_t tj = (r + 31) / 32;
+  for (int64_t t = blockIdx.x; t < tr * tj; t += gridDim.x) {
+    const int64_t row0 = (t % tr) * 32;
+    const int j0 = static_cast<int>(t / tr) * 32;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rl = warp + 8 * i;
+      const int64_t row = row0 + rl;
+      const int j = j0 + lane;
+      tile[rl][lane] = (row < rows && j < r) ? sum_splits(part + row * ld_part + j, splits, part_stride) : 0.f;
     }
-    float s = 0.f;
-    for (int t = 0; t < splits; ++t) s += part[t * part_stride + row * ld_part + j];
-    s = __fmul_rn(scale, s);
-    const int64_t o = transpose ? (j * rows + row) : (row * r + j);
-    out[o] = accumulate ? (out[o] + s) : s;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int jl = warp + 8 * i;
+      const int j = j0 + jl;
+      const int64_t row = row0 + lane;
+      if (j < r && row < rows) {
+        const float s = __fmul_rn(scale, tile[lane][jl]);
+        const int64_t o = static_cast<int64_t>(j) * rows + row;
+        out[o] = accumulate ? (out[o] + s) : s;
+      }
+    }
+    __syncthreads();
   }
 }
 
 cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_stride, int64_t rows, int32_t r,
                                  int32_t ld_part, float scale, float* out, int transpose, int accumulate,
                                  cudaStream_t st) {
-  grad_finalize_kernel<<<blocks_for(rows * r, 256), 256, 0, st>>>(part, splits, part_stride, rows, r, ld_part,
-                                                                   scale, out, transpose, accumulate);
-  count_launches(1);
-  return cudaGetLastError();
+  if (transpose) {
+    const int64_t tiles = ((rows + 31) / 32) * ((r + 31) / 32);
+    const int grid = static_cast<int>(tiles < 148 * 8 ? tiles : 148 * 8);
+    return launch_pdl(grad_finalize_t_kernel, grid < 1 ? 1 : grid, 256, 0, st, 1, part, splits, part_stride, rows,
+                      static_cast<int>(r), static_cast<int>(ld_part), scale, out, accumulate);
+  }
+  return launch_pdl(grad_finalize_kernel, blocks_for(rows * r, 256), 256, 0, st, 1, part, splits, part_stride, rows,
+                    static_cast<int>(r), static_cast<int>(ld_part), scale, out, accumulate);
 }
 
 // out[row, col] (+)= sum_t part[t][row][col], 4 columns per thread.
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t part_stride, int64_t rows,
                                      int64_t cols, int64_t ld_part, void* __restrict__ out, int out_bf16,
                                      int accumulate) {
+  griddep_enter();
   // eight consecutive columns per thread (cols % 8 == 0): two 16-byte partial loads per
   // split and one 16-byte BF16 (or two fp32) accesses of the output
   const int64_t c8 = cols / 8;
@@ -116,12 +152,24 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
     const int64_t row = idx / c8;
     const int64_t col = (idx - row * c8) * 8;
     float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int t = 0; t < splits; ++t) {
-      const float4* src = reinterpret_cast<const float4*>(part + t * part_stride + row * ld_part + col);
-      const float4 a = __ldcs(src);
-      const float4 b = __ldcs(src + 1);
-      s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
-      s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
+    // four splits' loads in flight at a time, added in split order
+    for (int t0 = 0; t0 < splits; t0 += 4) {
+      float4 a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u < splits) {
+          const float4* src = reinterpret_cast<const float4*>(part + (t0 + u) * part_stride + row * ld_part + col);
+          a[u] = __ldcs(src);
+          b[u] = __ldcs(src + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (t0 + u < splits) {
+          s[0] += a[u].x; s[1] += a[u].y; s[2] += a[u].z; s[3] += a[u].w;
+          s[4] += b[u].x; s[5] += b[u].y; s[6] += b[u].z; s[7] += b[u].w;
+        }
+      }
     }
     if (out_bf16) {
       uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row * cols + col);
@@ -156,10 +204,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
 cudaError_t launch_splitk_reduce(const float* part, int splits, int64_t part_stride, int64_t rows, int64_t cols,
                                  int64_t ld_part, void* out, int out_bf16, int accumulate, cudaStream_t st) {
   if (cols % 8 != 0 || ld_part % 8 != 0) return cudaErrorInvalidValue;
-  splitk_reduce_kernel<<<blocks_for(rows * (cols / 8), 256), 256, 0, st>>>(part, splits, part_stride, rows, cols,
-                                                                            ld_part, out, out_bf16, accumulate);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(splitk_reduce_kernel, blocks_for(rows * (cols / 8), 256), 256, 0, st, 1, part, splits,
+                    part_stride, rows, cols, ld_part, out, out_bf16, accumulate);
 }
 
 // ---------------------------------------------------------------------------
@@ -190,9 +236,9 @@ __global__ void __launch_bounds__(kSmallThreads) lora_down_small_kernel(const ui
                                                                        uint16_t* __restrict__ out_scaled) {
   __shared__ float red[kSmallThreads / 32][MMAX];
   __shared__ float slice_sum[MMAX];
-  // the fused GEMM launched after this kernel may start streaming its weight now; it
-  // waits for this grid before it reads bf16(scale * U)
-  griddep_launch_dependents();
+  // the fused GEMM launched after this kernel may start streaming its weight once every
+  // CTA is past this point; it waits for this grid before it reads bf16(scale * U)
+  griddep_enter();
   const int j = blockIdx.x / kSmallSlices;
   const uint32_t slice = cluster_ctarank();
   const int64_t slice_len = ((k / 8 + kSmallSlices - 1) / kSmallSlices) * 8;
@@ -256,26 +302,13 @@ __global__ void __launch_bounds__(kSmallThreads) lora_down_small_kernel(const ui
 cudaError_t launch_lora_down_small(const uint16_t* X, int64_t m, int64_t k, const uint16_t* A, int32_t r,
                                    int32_t r_pad, float scale, float* U32, uint16_t* sU, cudaStream_t st, float pre) {
   if (m > 64 || k % 8 != 0) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(r_pad * kSmallSlices), 1, 1);
-  cfg.blockDim = dim3(kSmallThreads, 1, 1);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kSmallSlices;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   const int mi = static_cast<int>(m);
-  cudaError_t e = (m <= 16)
-                      ? cudaLaunchKernelEx(&cfg, lora_down_small_kernel<16>, X, mi, k, A, static_cast<int>(r),
-                                           static_cast<int>(r_pad), scale, pre, U32, sU)
-                      : cudaLaunchKernelEx(&cfg, lora_down_small_kernel<64>, X, mi, k, A, static_cast<int>(r),
-                                           static_cast<int>(r_pad), scale, pre, U32, sU);
-  count_launches(1);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  const int grid = static_cast<int>(r_pad) * kSmallSlices;
+  if (m <= 16)
+    return launch_pdl(lora_down_small_kernel<16>, grid, kSmallThreads, 0, st, kSmallSlices, X, mi, k, A,
+                      static_cast<int>(r), static_cast<int>(r_pad), scale, pre, U32, sU);
+  return launch_pdl(lora_down_small_kernel<64>, grid, kSmallThreads, 0, st, kSmallSlices, X, mi, k, A,
+                    static_cast<int>(r), static_cast<int>(r_pad), scale, pre, U32, sU);
 }
 
 // ---------------------------------------------------------------------------
@@ -361,6 +394,7 @@ __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf
 
 __global__ void silu_gate_fwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ u,
                                      uint16_t* __restrict__ h, int64_t count) {
+  griddep_enter();
   const int64_t n8 = count / 8;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -386,6 +420,7 @@ __global__ void silu_gate_fwd_kernel(const uint16_t* __restrict__ g, const uint1
 __global__ void silu_gate_bwd_kernel(const uint16_t* __restrict__ dh, const uint16_t* __restrict__ g,
                                      const uint16_t* __restrict__ u, uint16_t* __restrict__ dg,
                                      uint16_t* __restrict__ du, int64_t count) {
+  griddep_enter();
   const int64_t n8 = count / 8;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -423,16 +458,13 @@ __global__ void silu_gate_bwd_kernel(const uint16_t* __restrict__ dh, const uint
 
 cudaError_t launch_silu_gate_fwd(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t count,
                                  cudaStream_t st) {
-  silu_gate_fwd_kernel<<<blocks_for((count + 7) / 8, 256), 256, 0, st>>>(g, u, h, count);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(silu_gate_fwd_kernel, blocks_for((count + 7) / 8, 256), 256, 0, st, 1, g, u, h, count);
 }
 
 cudaError_t launch_silu_gate_bwd(const uint16_t* dh, const uint16_t* g, const uint16_t* u, uint16_t* dg,
                                  uint16_t* du, int64_t count, cudaStream_t st) {
-  silu_gate_bwd_kernel<<<blocks_for((count + 7) / 8, 256), 256, 0, st>>>(dh, g, u, dg, du, count);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(silu_gate_bwd_kernel, blocks_for((count + 7) / 8, 256), 256, 0, st, 1, dh, g, u, dg, du,
+                    count);
 }
 
 }  // namespace qlora

@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     }
     fence_mbar_init();
   }
+  griddep_enter();
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -486,8 +487,7 @@ static cudaError_t launch_cfg(const GemmParams& p, const GemmMaps& maps, int gri
       attr_set[dev] = true;
     }
   }
-  qlora_gemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p, maps);
-  return cudaGetLastError();
+  return launch_pdl(qlora_gemm_kernel<C>, grid, C::kThreads, C::kSmemBytes, st, 1, p, maps);
 }
 
 using CfgDownK = GemmCfg<64, 6, false, kB_TmaK, false, false>;
@@ -520,9 +520,7 @@ static cudaError_t launch_gemm_impl(GemmKind kind, const GemmParams& p, const Ge
 }
 
 cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps, int grid, cudaStream_t st) {
-  const cudaError_t e = launch_gemm_impl(kind, p, maps, grid, st);
-  count_launches(1);
-  return e;
+  return launch_gemm_impl(kind, p, maps, grid, st);
 }
 
 }  // namespace qlora

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_mbar_init();
   }
+  griddep_enter();
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -355,8 +356,8 @@ cudaError_t launch_merge_impl(const MergeParams& p, const MergeMaps& m, int grid
       attr_set[dev] = true;
     }
   }
-  qlora_merge_kernel<kF32><<<grid, kThreads, MergeSmem<kF32>::kBytes, st>>>(p, m.b, m.a, m.codes, m.out);
-  return cudaGetLastError();
+  return launch_pdl(qlora_merge_kernel<kF32>, grid, kThreads, MergeSmem<kF32>::kBytes, st, 1, p, m.b, m.a, m.codes,
+                    m.out);
 }
 
 }  // namespace
@@ -364,9 +365,7 @@ cudaError_t launch_merge_impl(const MergeParams& p, const MergeMaps& m, int grid
 int merge_tile_cols() { return kMergeBN; }
 
 cudaError_t launch_merge(const MergeParams& p, const MergeMaps& maps, int grid, bool out_f32, cudaStream_t st) {
-  const cudaError_t e = out_f32 ? launch_merge_impl<true>(p, maps, grid, st) : launch_merge_impl<false>(p, maps, grid, st);
-  count_launches(1);
-  return e;
+  return out_f32 ? launch_merge_impl<true>(p, maps, grid, st) : launch_merge_impl<false>(p, maps, grid, st);
 }
 
 }  // namespace qlora

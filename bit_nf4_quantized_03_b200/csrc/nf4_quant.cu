@@ -453,27 +453,6 @@ __global__ void __launch_bounds__(256, 3) nf4_dequantize_kernel(const uint8_t* _
 // launchers
 // ---------------------------------------------------------------------------
 
-// Launch with programmatic dependent launch allowed: the kernel may be scheduled while
-// the one before it on the stream finishes; each kernel here waits (griddepcontrol.wait)
-// before it reads anything that kernel may write.
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, int smem, cudaStream_t st,
-                              Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(static_cast<unsigned>(block), 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  count_launches(1);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-  return e != cudaSuccess ? e : cudaGetLastError();
-}
-
 template <typename K>
 static cudaError_t set_smem_once(K kernel, int bytes, bool* done) {
   int dev = 0;
@@ -509,7 +488,7 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   if (!dq) {
     e = set_smem_once(nf4_quantize_kernel<false>, kQSmem, smem_set[0]);
     if (e != cudaSuccess) return e;
-    return launch_pdl(nf4_quantize_kernel<false>, grid, 256, kQSmem, st, wmap, W, n_elem, bk, codes, scale_bf16,
+    return launch_pdl(nf4_quantize_kernel<false>, grid, 256, kQSmem, st, 1, wmap, W, n_elem, bk, codes, scale_bf16,
                       static_cast<float*>(nullptr), static_cast<double*>(nullptr));
   }
   const QuantWsLayout L = quant_ws_layout(n_elem);
@@ -518,18 +497,18 @@ cudaError_t launch_quantize(const float* W, int64_t n_elem, const Nf4Table& tab,
   // stage 1 also writes one fp64 tree sum per chunk (the first levels of the fixed-order sum)
   e = set_smem_once(nf4_quantize_kernel<true>, kQSmem, smem_set[1]);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(nf4_quantize_kernel<true>, grid, 256, kQSmem, st, wmap, W, n_elem, bk, codes,
+  e = launch_pdl(nf4_quantize_kernel<true>, grid, 256, kQSmem, st, 1, wmap, W, n_elem, bk, codes,
                  static_cast<uint16_t*>(nullptr), absmax, part_a);
   if (e != cudaSuccess) return e;
   // the rest of the tree and the mean (one CTA), then the E4M3 pass
-  e = launch_pdl(dq_mean_kernel, 1, 1024, 0, st, static_cast<const double*>(part_a), nchunks, nblk, dq_mean);
+  e = launch_pdl(dq_mean_kernel, 1, 1024, 0, st, 1, static_cast<const double*>(part_a), nchunks, nblk, dq_mean);
   if (e != cudaSuccess) return e;
   const int64_t nb2 = (nblk + 255) / 256;
   // enough CTAs that each takes at most kFinishPer 256-blocks, at least one per SM when there is work
   int64_t g2 = (nb2 + kFinishPer - 1) / kFinishPer;
   if (g2 < num_sms) g2 = nb2 < num_sms ? nb2 : num_sms;
   const int grid2 = static_cast<int>(g2);
-  return launch_pdl(dq_finish_kernel, grid2, 256, 0, st, static_cast<const float*>(dq_mean),
+  return launch_pdl(dq_finish_kernel, grid2, 256, 0, st, 1, static_cast<const float*>(dq_mean),
                     static_cast<const float*>(absmax), nblk, scale_fp8, dq_scale);
 }
 
@@ -542,7 +521,7 @@ cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t 
   const int64_t nchunks = (nfull + kDChunk - 1) / kDChunk;
   int64_t grid = nchunks < 3LL * num_sms ? nchunks : 3LL * num_sms;
   if (grid < 1) grid = 1;
-  return launch_pdl(nf4_dequantize_kernel, static_cast<int>(grid), 256, kDSmem, st, codes, ss, n_elem, tab, out);
+  return launch_pdl(nf4_dequantize_kernel, static_cast<int>(grid), 256, kDSmem, st, 1, codes, ss, n_elem, tab, out);
 }
 
 }  // namespace qlora

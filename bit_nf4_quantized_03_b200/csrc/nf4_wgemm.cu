@@ -191,6 +191,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     }
     fence_mbar_init();
   }
+  // an early launch streams the weight before the grid before it has finished (the
+  // producer waits before the extension); otherwise nothing is touched before it has
+  if (!p.early) griddep_enter();
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -630,6 +633,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     }
     fence_mbar_init();
   }
+  griddep_enter();
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::kTmemCols);
     tmem_relinquish_pair();
@@ -915,19 +919,7 @@ static cudaError_t launch_pcfg(const GemmParams& p, const WMaps& maps, int grid,
     }
   }
   if (grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(C::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, qlora_wgemm_pair_kernel<C>, p, maps);
+  return launch_pdl(qlora_wgemm_pair_kernel<C>, grid, C::kThreads, C::kSmemBytes, st, 2, p, maps);
 }
 
 // CTA pairs of the 256-token kernel that fit on the device at once (one CTA per SM).
@@ -980,21 +972,9 @@ static cudaError_t launch_wcfg(const GemmParams& p, const WMaps& maps, int grid,
       attr_set[dev] = true;
     }
   }
-  if (!early) {
-    qlora_wgemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p, maps);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(C::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, qlora_wgemm_kernel<C>, p, maps);
+  GemmParams q = p;
+  q.early = early ? 1 : 0;
+  return launch_pdl(qlora_wgemm_kernel<C>, grid, C::kThreads, C::kSmemBytes, st, 1, q, maps);
 }
 
 int wgemm_box_rows(int bn) { return bn >= 256 ? 128 : bn; }   // a CTA pair loads half of each 256-token tile
@@ -1042,7 +1022,6 @@ cudaError_t launch_wgemm(bool bwd, int bn, const GemmParams& p, const WMaps& map
     }
   }
   if (timed) timing_record(st, false, algo_flops);
-  count_launches(1);
   return e;
 }
 

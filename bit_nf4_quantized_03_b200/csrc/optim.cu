@@ -42,6 +42,7 @@ __device__ __forceinline__ void adam1(float& p, float g, float& m, float& v, con
 __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
                                                     float* __restrict__ m, float* __restrict__ v,
                                                     uint16_t* __restrict__ p_bf16, int64_t count, AdamCoef c) {
+  griddep_enter();
   const int64_t n4 = count / 4;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
@@ -91,9 +92,7 @@ cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, uint16_t*
   int64_t blocks = (count / 4 + 255) / 256;
   if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
   if (blocks < 1) blocks = 1;
-  adamw_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(p, g, m, v, p_bf16, count, c);
-  count_launches(1);
-  return cudaGetLastError();
+  return launch_pdl(adamw_kernel, static_cast<int>(blocks), 256, 0, st, 1, p, g, m, v, p_bf16, count, c);
 }
 
 }  // namespace qlora

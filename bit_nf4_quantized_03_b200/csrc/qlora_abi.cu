@@ -336,7 +336,8 @@ bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint
 // Low-rank product U (or G): partial GEMM over the reduction, then finalize.
 int run_lora_down(const Plan& P, bool b_mn, const uint16_t* act, int64_t m, int64_t red, const uint16_t* adapter,
                   int32_t r, float scale, char* ws, float* out_f32, uint16_t* out_scaled, uint16_t* out_hi,
-                  uint16_t* out_lo, cudaStream_t st, float pre = 1.0f) {
+                  uint16_t* out_lo, cudaStream_t st, float pre = 1.0f, const float* extra_src = nullptr,
+                  uint16_t* extra_hi = nullptr, uint16_t* extra_lo = nullptr) {
   const Split sp = b_mn ? P.g : P.u;
   GemmParams p = base_params(m, P.r_pad, P.r_pad, b_mn ? cdiv(red, 64) : red / 64, sp);
   p.out = ws + P.off_part;
@@ -355,7 +356,7 @@ int run_lora_down(const Plan& P, bool b_mn, const uint16_t* act, int64_t m, int6
   cudaError_t e = launch_gemm(b_mn ? P.down_mn : P.down_k, p, maps, grid_of(p), st);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   e = launch_lora_finalize(static_cast<const float*>(p.out), sp.splits, p.part_stride, m, r, P.r_pad, scale,
-                           out_f32, out_scaled, out_hi, out_lo, st, pre);
+                           out_f32, out_scaled, out_hi, out_lo, st, pre, extra_src, extra_hi, extra_lo);
   return cuda_status(e);
 }
 
@@ -653,13 +654,13 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
   uint16_t* u_lo = reinterpret_cast<uint16_t*>(wsb + P.off_lo_a);
   const int acc_grads = (flags & QLORA_BWD_ACCUMULATE_GRADS) ? 1 : 0;
 
-  // G = dY B: bf16(s G) for the dX extension, hi/lo bf16 for dA
-  int rc = run_lora_down(P, true, dY, m, n, B, r, s, wsb, nullptr, sG, g_hi, g_lo, st);
+  // G = dY B: bf16(s G) for the dX extension, hi/lo bf16 for dA; the saved U's hi/lo bf16
+  // split for dB comes out of the same finalize launch
+  int rc = run_lora_down(P, true, dY, m, n, B, r, s, wsb, nullptr, sG, g_hi, g_lo, st, 1.0f, U_saved,
+                         U_saved != nullptr ? u_hi : nullptr, U_saved != nullptr ? u_lo : nullptr);
   if (rc != QLORA_OK) return rc;
-  // U = X A^T as hi/lo bf16 for dB (recomputed when not saved)
-  if (U_saved != nullptr) {
-    if (launch_split_hilo(U_saved, m, r, P.r_pad, u_hi, u_lo, st) != cudaSuccess) return QLORA_ERR_CUDA;
-  } else {
+  // U = X A^T as hi/lo bf16 for dB, recomputed when not saved
+  if (U_saved == nullptr) {
     rc = run_lora_down(P, false, Xl, m, k, A, r, s, wsb, nullptr, nullptr, u_hi, u_lo, st, D.keep);
     if (rc != QLORA_OK) return rc;
   }

@@ -188,6 +188,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // side, a grid launched after this one with that allowance may start now.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+// Programmatic dependent launch, at a kernel's start: wait until the grid before this one
+// on the stream has completed and its writes are visible, then allow the grid after this
+// one to be scheduled (it waits in turn before it touches memory). A no-op for a launch
+// without the programmatic attribute.
+__device__ __forceinline__ void griddep_enter() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y) {

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "qlora_device.cuh"
 
 namespace qlora {
@@ -81,6 +83,10 @@ struct GemmParams {
   // masked modes: bit (row * ld_out + col) of `mask` (bit e % 8 of byte e / 8) keeps the element
   const uint8_t* mask;
   float keep_scale;
+  // single-CTA weight GEMM only (set by launch_wgemm): 1 = started before the grid that
+  // writes the low-rank operand has finished; only the producer waits, before its first
+  // extension load
+  int32_t early;
 };
 
 struct GemmMaps {
@@ -110,6 +116,37 @@ cudaError_t launch_gemm(GemmKind kind, const GemmParams& p, const GemmMaps& maps
 void count_launches(int n);
 bool timing_active();
 void timing_record(cudaStream_t st, bool start, double flops);
+
+// Launch with programmatic dependent launch allowed: the grid may be scheduled while the
+// grid before it on the stream finishes. Every kernel of the library starts with
+// griddep_enter() (or, where stated, waits later), so it reads and writes nothing before
+// the grid before it has completed, and the grid after it is scheduled only once all of
+// this grid's CTAs are past that wait. `cluster_x` > 1 adds a cluster dimension.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                              int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(block), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int na = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    na = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  count_launches(1);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 // ------------------------------------------------------- weight-operand GEMM
 // (nf4_wgemm.cu) D^T[features, tokens] with the dequantized weight as the
@@ -157,12 +194,12 @@ cudaError_t launch_merge(const MergeParams& p, const MergeMaps& maps, int grid, 
 
 // ------------------------------------------------------------- elementwise
 // U = pre * (sum of the split partials); writes fp32 U, bf16(scale * U), hi/lo bf16 of U (each nullable).
+// extra_src (nullable): a second fp32 [rows, r] matrix split into hi/lo bf16 [rows, r_pad] in the same launch.
 cudaError_t launch_lora_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
                                  int32_t r, int32_t r_pad, float scale, float* out_f32,
                                  uint16_t* out_scaled_bf16, uint16_t* out_hi, uint16_t* out_lo,
-                                 cudaStream_t st, float pre = 1.0f);
-cudaError_t launch_split_hilo(const float* src, int64_t rows, int32_t r, int32_t r_pad, uint16_t* hi,
-                              uint16_t* lo, cudaStream_t st);
+                                 cudaStream_t st, float pre = 1.0f, const float* extra_src = nullptr,
+                                 uint16_t* extra_hi = nullptr, uint16_t* extra_lo = nullptr);
 cudaError_t launch_grad_finalize(const float* part, int splits, int64_t part_stride, int64_t rows,
                                  int32_t r, int32_t ld_part, float scale, float* out, int transpose,
                                  int accumulate, cudaStream_t st);
