@@ -364,6 +364,8 @@ class Workload:
         self.host_grads = torch.empty(self.grads.shape, dtype=f32).pin_memory()
         ws = max(max(q.qlora_linear_workspace_bytes(M, n, k, RANK_R),
                      q.qlora_linear_workspace_bytes(M_SMALL, n, k, RANK_R)) for _, n, k in LAYERS)
+        ws = max(ws, q.qlora_linear_group_workspace_bytes(M, [H, H, H], H, RANK_R),
+                 q.qlora_linear_group_workspace_bytes(M, [I, I], H, RANK_R))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.host.values())
@@ -378,6 +380,14 @@ class Workload:
         flags = q.QLORA_BWD_ACCUMULATE_DX if acc_dx else 0
         q.qlora_linear_bwd(self.w[nm], X, dY, self.A[nm], self.B[nm], RANK_R, ALPHA, self.U[nm], dX,
                            q.QLORA_DTYPE_BF16, self.dA[nm], self.dB[nm], flags, self.ws)
+
+    def _bwd_group(self, names, X, dYs, dX):
+        """Backward of the layers in `names`, which share the input X: one fused dX GEMM."""
+        q = self.q
+        q.qlora_linear_bwd_group([self.w[nm] for nm in names], X, list(dYs), [self.A[nm] for nm in names],
+                                 [self.B[nm] for nm in names], RANK_R, ALPHA, [self.U[nm] for nm in names], dX,
+                                 q.QLORA_DTYPE_BF16, [self.dA[nm] for nm in names], [self.dB[nm] for nm in names],
+                                 0, self.ws)
 
     def _inputs(self):
         """The input set, as a mapping whose lookup first makes the compute stream wait
@@ -403,12 +413,10 @@ class Workload:
         self._fwd("down_proj", self.h, self.y_mlp, self.U["down_proj"])
         self._bwd("down_proj", self.h, d["dy_mlp"], self.dh, False)
         q.qlora_silu_gate_bwd(self.dh, self.g, self.u, self.dg, self.du)
-        self._bwd("gate_proj", d["x_mlp"], self.dg, self.dx_mlp, False)
-        self._bwd("up_proj", d["x_mlp"], self.du, self.dx_mlp, True)
+        self._bwd_group(("gate_proj", "up_proj"), d["x_mlp"], (self.dg, self.du), self.dx_mlp)
         self._bwd("o_proj", d["x_o"], d["dy_o"], self.dx_o, False)
-        self._bwd("q_proj", d["x_attn"], d["dy_q"], self.dx_attn, False)
-        self._bwd("k_proj", d["x_attn"], d["dy_k"], self.dx_attn, True)
-        self._bwd("v_proj", d["x_attn"], d["dy_v"], self.dx_attn, True)
+        self._bwd_group(("q_proj", "k_proj", "v_proj"), d["x_attn"], (d["dy_q"], d["dy_k"], d["dy_v"]),
+                        self.dx_attn)
         for nm, _, _ in LAYERS:
             x = d["h16"] if nm == "down_proj" else d["x16"]
             self._fwd(nm, x, self.y16[nm], None)
@@ -625,8 +633,8 @@ def _seven_b_components(q, synth, torch, dev, flush, peaks, out):
     Us = {nm: e(M, RANK_R, dt=f32) for nm in lay}
     dAs = {nm: e(RANK_R, lay[nm][0].k, dt=f32) for nm in lay}
     dBs = {nm: e(lay[nm][0].n, RANK_R, dt=f32) for nm in lay}
-    ws = torch.empty(max(q.qlora_linear_workspace_bytes(M, I, H, RANK_R),
-                         q.qlora_linear_workspace_bytes(M, H, I, RANK_R)), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(q.qlora_linear_workspace_bytes(M, I, H, RANK_R), q.qlora_linear_workspace_bytes(M, H, I, RANK_R),
+                         q.qlora_linear_group_workspace_bytes(M, [I, I], H, RANK_R)), dtype=torch.uint8, device=dev)
 
     def fwd(nm, x, yy):
         qw_, a_, b_ = lay[nm]
@@ -644,8 +652,11 @@ def _seven_b_components(q, synth, torch, dev, flush, peaks, out):
         fwd("down", h, y)
         bwd("down", h, dY, dh, False)
         q.qlora_silu_gate_bwd(dh, g, u, dg, du)
-        bwd("gate", X, dg, dx, False)
-        bwd("up", X, du, dx, True)
+        # gate and up read the same X: one grouped backward forms dX
+        gu = ("gate", "up")
+        q.qlora_linear_bwd_group([lay[nm][0] for nm in gu], X, [dg, du], [lay[nm][1] for nm in gu],
+                                 [lay[nm][2] for nm in gu], RANK_R, ALPHA, [Us[nm] for nm in gu], dx,
+                                 q.QLORA_DTYPE_BF16, [dAs[nm] for nm in gu], [dBs[nm] for nm in gu], 0, ws)
     for _ in range(2):
         mlp()
     ms = graph_time(mlp, 3, flush)

@@ -20,14 +20,20 @@ BOUNDS_CHECK = os.environ.get("QLORA_BOUNDS_CHECK", "") not in ("", "0")
 LIB_PATH = os.path.join(_PKG, "libqlora_bounds.so" if BOUNDS_CHECK else "libqlora.so")
 
 QLORA_OK = 0
+QLORA_ERR_INVALID = 1
+QLORA_ERR_UNSUPPORTED = 2
+QLORA_ERR_CUDA = 3
+QLORA_ERR_WORKSPACE = 4
+QLORA_ERR_DEVICE = 5
+QLORA_ERR_BOUNDS = 6
 QLORA_SCALE_BF16 = 0
 QLORA_SCALE_DQ_FP8 = 1
 QLORA_DTYPE_BF16 = 0
 QLORA_DTYPE_FP32 = 1
 QLORA_BWD_ACCUMULATE_GRADS = 1
 QLORA_BWD_ACCUMULATE_DX = 2
-BLOCKSIZE = 64
-DQ_BLOCKSIZE = 256
+QLORA_BLOCKSIZE = BLOCKSIZE = 64
+QLORA_DQ_BLOCKSIZE = DQ_BLOCKSIZE = 256
 
 # every symbol include/qlora.h declares
 EXPORTED = (
@@ -39,7 +45,7 @@ EXPORTED = (
     "qlora_nf4_quantize_noalloc", "qlora_selftest_wait_timeout", "qlora_lora_merge",
     "qlora_linear_workspace_bytes_ex", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
     "qlora_adamw_step", "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch",
-    "qlora_expand_rate", "qlora_bounds_site",
+    "qlora_expand_rate", "qlora_bounds_site", "qlora_linear_bwd_group", "qlora_linear_group_workspace_bytes",
 )
 
 
@@ -126,6 +132,9 @@ def lib() -> ctypes.CDLL:
         "qlora_bounds_site": (ctypes.c_int, []),
         "qlora_lora_merge": (ctypes.c_int, [pw, vp, vp, i32, f32, vp, i32, vp]),
         "qlora_linear_workspace_bytes_ex": (sz, [i64, i64, i64, i32, pd]),
+        "qlora_linear_bwd_group": (ctypes.c_int, [i32, vp, vp, vp, i64, vp, vp, i32, f32, vp, vp, i32, vp, vp, i32,
+                                                  vp, sz, vp]),
+        "qlora_linear_group_workspace_bytes": (sz, [i32, i64, vp, i64, i32]),
         "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWConfig), vp]),
         "qlora_paged_alloc": (ctypes.c_int, [sz, ctypes.POINTER(ctypes.c_void_p)]),
         "qlora_paged_free": (ctypes.c_int, [vp]),
@@ -294,6 +303,33 @@ def qlora_linear_bwd_ex(w: QuantizedWeight, X, dY, A, B, r: int, alpha: float, U
                                    _ptr(U_saved), _ptr(dX), dx_dtype, _ptr(dA), _ptr(dB), flags, _dref(drop),
                                    _ptr(ws), ws_bytes, _stream(stream))
     _check(rc, "qlora_linear_bwd_ex")
+
+
+def _ptr_array(items):
+    """A C array of device addresses (None entries stay NULL)."""
+    return (ctypes.c_void_p * len(items))(*[_ptr(t) for t in items])
+
+
+def qlora_linear_group_workspace_bytes(m: int, ns, k: int, r: int) -> int:
+    arr = (ctypes.c_int64 * len(ns))(*[int(n) for n in ns])
+    return int(lib().qlora_linear_group_workspace_bytes(len(ns), m, ctypes.addressof(arr), k, r))
+
+
+def qlora_linear_bwd_group(ws_list, X, dYs, As, Bs, r: int, alpha: float, U_saved, dX, dx_dtype: int,
+                           dAs, dBs, flags: int = 0, ws=None, stream=None):
+    """Backward of len(ws_list) layers sharing the input X: dX (+)= sum of the layers' terms,
+    each layer's dA, dB as qlora_linear_bwd gives them."""
+    count = len(ws_list)
+    wp = (ctypes.POINTER(NF4Weight) * count)(*[ctypes.pointer(w.struct) for w in ws_list])
+    dy, a, b, da, db = (_ptr_array(t) for t in (dYs, As, Bs, dAs, dBs))
+    us = None if U_saved is None else _ptr_array(U_saved)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = lib().qlora_linear_bwd_group(count, ctypes.addressof(wp), _ptr(X), ctypes.addressof(dy), X.shape[0],
+                                      ctypes.addressof(a), ctypes.addressof(b), r, float(alpha),
+                                      None if us is None else ctypes.addressof(us), _ptr(dX), dx_dtype,
+                                      ctypes.addressof(da), ctypes.addressof(db), flags, _ptr(ws), ws_bytes,
+                                      _stream(stream))
+    _check(rc, "qlora_linear_bwd_group")
 
 
 def qlora_adamw_step(param, grad, m, v, param_bf16, count: int, cfg: AdamWConfig, stream=None):

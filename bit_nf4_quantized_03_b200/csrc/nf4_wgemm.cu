@@ -81,7 +81,12 @@ __device__ __forceinline__ void wdecode(const GemmParams& p, int u, int& mb, int
   int kt1 = kt0 + p.k_per_split;
   if (kt1 > p.k_tiles) kt1 = p.k_tiles;
   nmain = kt1 - kt0;
-  next = (split == 0) ? p.ext_tiles : 0;
+  next = (split == 0) ? p.ext_tiles * (p.groups > 1 ? p.groups : 1) : 0;   // every layer's extension
+}
+
+// Layer of main K step kt in a grouped GEMM (0 for one layer).
+__device__ __forceinline__ int wlayer(const GemmParams& p, int kt) {
+  return (p.groups > 1) ? (kt >= p.k_begin[1] ? 1 : 0) + ((p.groups > 2 && kt >= p.k_begin[2]) ? 1 : 0) : 0;
 }
 
 __device__ __forceinline__ void st_shared_v4_w(uint32_t addr, uint4 v) {
@@ -206,10 +211,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&maps.act);
-      tma_prefetch_desc(&maps.codes);
-      tma_prefetch_desc(&maps.a2);
-      tma_prefetch_desc(&maps.b2);
+      tma_prefetch_desc(&maps.act[0]);
+      tma_prefetch_desc(&maps.codes[0]);
+      tma_prefetch_desc(&maps.a2[0]);
+      tma_prefetch_desc(&maps.b2[0]);
       int stage = 0;
       uint32_t ph = 0;
       uint32_t pending = 0, pend_par = 0;
@@ -235,30 +240,30 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_arrive_expect_tx(bar, C::kRBytes + C::kBTile);
             if (C::Bwd) {
               if (tma_start_ok(mb * 64, kt * 64, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 10))
-                tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, mb * 64, kt * 64);
+                tma_load_2d(sR + stage * C::kRBytes, &maps.codes[0], bar, mb * 64, kt * 64);
             } else if (tma_start_ok(kt * 32, mb * 128, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 11)) {
-              tma_load_2d(sR + stage * C::kRBytes, &maps.codes, bar, kt * 32, mb * 128);
+              tma_load_2d(sR + stage * C::kRBytes, &maps.codes[0], bar, kt * 32, mb * 128);
             }
 #pragma unroll
             for (int t = 0; t < C::NAcc; ++t)
-              if (tma_start_ok(kt * 64, nb * C::TOK + t * C::BN, 2, C::Bwd ? p.w_rows : p.w_kblocks * 64,
+              if (tma_start_ok(kt * 64, nb * C::TOK + t * C::BN, 2, C::Bwd ? p.w_rows[0] : p.w_kblocks * 64,
                                b_dst + t * (C::BN * 128), 12))
-                tma_load_2d(b_dst + t * (C::BN * 128), &maps.act, bar, kt * 64, nb * C::TOK + t * C::BN);
+                tma_load_2d(b_dst + t * (C::BN * 128), &maps.act[0], bar, kt * 64, nb * C::TOK + t * C::BN);
           } else {
             const int e = i - nmain;
             mbar_arrive_expect_tx(bar, C::kATile + C::kBTile);
             if (C::Bwd) {
               if (tma_start_ok(mb * 128, e * 64, 2, p.w_kblocks * 64, a_dst, 13))
-                tma_load_2d(a_dst, &maps.a2, bar, mb * 128, e * 64);
+                tma_load_2d(a_dst, &maps.a2[0], bar, mb * 128, e * 64);
               if (tma_start_ok(mb * 128 + 64, e * 64, 2, p.w_kblocks * 64, a_dst + 8192, 14))
-                tma_load_2d(a_dst + 8192, &maps.a2, bar, mb * 128 + 64, e * 64);
+                tma_load_2d(a_dst + 8192, &maps.a2[0], bar, mb * 128 + 64, e * 64);
             } else if (tma_start_ok(e * 64, mb * 128, 2, p.ext_tiles * 64, a_dst, 15)) {
-              tma_load_2d(a_dst, &maps.a2, bar, e * 64, mb * 128);
+              tma_load_2d(a_dst, &maps.a2[0], bar, e * 64, mb * 128);
             }
 #pragma unroll
             for (int t = 0; t < C::NAcc; ++t)
               if (tma_start_ok(e * 64, nb * C::TOK + t * C::BN, 2, p.ext_tiles * 64, b_dst + t * (C::BN * 128), 16))
-                tma_load_2d(b_dst + t * (C::BN * 128), &maps.b2, bar, e * 64, nb * C::TOK + t * C::BN);
+                tma_load_2d(b_dst + t * (C::BN * 128), &maps.b2[0], bar, e * 64, nb * C::TOK + t * C::BN);
           }
           pending |= (1u << stage);
           pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // Backward: thread = (W row i of the 64-row K step, 64-column block c of the tile).
     const int grp = (warp - 6) >> 2;
     const int gt = threadIdx.x - 192 - 128 * grp;    // 0..127
-    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
+    const float mean = (p.scales[0].dq_mean != nullptr) ? __ldg(p.scales[0].dq_mean) : 0.f;
     const int i_mn = gt & 63;
     const int c_mn = gt >> 6;
     uint32_t r_off0, r_off1, a_off;
@@ -386,7 +391,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         int64_t wrow, kb;
         if (!C::Bwd) { wrow = static_cast<int64_t>(mb) * 128 + gt; kb = kt; }
         else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(mb) * 2 + c_mn; }
-        valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
+        valid = (wrow < p.w_rows[0]) && (kb < p.w_kblocks);
         return wrow * p.w_kblocks + kb;
       };
       // scale prefetch: own K steps are every G-th step; keep four of them in flight
@@ -394,13 +399,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       {
         bool v;
         int64_t bb = block_of(first, v);
-        if (first < nmain && v) r0 = load_raw_scale(p.scales, bb);
+        if (first < nmain && v) r0 = load_raw_scale(p.scales[0], bb);
         bb = block_of(first + G, v);
-        if (first + G < nmain && v) r1 = load_raw_scale(p.scales, bb);
+        if (first + G < nmain && v) r1 = load_raw_scale(p.scales[0], bb);
         bb = block_of(first + 2 * G, v);
-        if (first + 2 * G < nmain && v) r2 = load_raw_scale(p.scales, bb);
+        if (first + 2 * G < nmain && v) r2 = load_raw_scale(p.scales[0], bb);
         bb = block_of(first + 3 * G, v);
-        if (first + 3 * G < nmain && v) r3 = load_raw_scale(p.scales, bb);
+        if (first + 3 * G < nmain && v) r3 = load_raw_scale(p.scales[0], bb);
       }
       for (int i = 0; i < nmain + next; ++i) {
         if (stage % G == grp) {
@@ -409,14 +414,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             block_of(i, valid);
             const int64_t b4 = block_of(i + 4 * G, v4);
             RawScale r4{0u, 0.f};
-            if (i + 4 * G < nmain && v4) r4 = load_raw_scale(p.scales, b4);
+            if (i + 4 * G < nmain && v4) r4 = load_raw_scale(p.scales[0], b4);
             if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
             const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
             if (valid) {
               const uint32_t rsrc = smem_u32(sR + stage * C::kRBytes);
               const uint4 w0 = ld_shared_v4_w(rsrc + r_off0);
               const uint4 w1 = ld_shared_v4_w(rsrc + r_off1);
-              const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales, r0, mean));
+              const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales[0], r0, mean));
               st_shared_v4_w(adst + ((0 ^ sw) << 4), nf4_lookup8(lut, w0.x));
               st_shared_v4_w(adst + ((1 ^ sw) << 4), nf4_lookup8(lut, w0.y));
               st_shared_v4_w(adst + ((2 ^ sw) << 4), nf4_lookup8(lut, w0.z));
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // its 64-block). Backward: thread = (W row i of the 64-row K step, 64-column block c
     // of the 128-column tile, half h).
     const int gt = threadIdx.x - 192;                 // 0..255
-    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
+    const float mean = (p.scales[0].dq_mean != nullptr) ? __ldg(p.scales[0].dq_mean) : 0.f;
     int row_f = 0, i_mn = 0, c_mn = 0, h;
     uint32_t r_off, a_off;
     int sw;
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         int64_t wrow, kb;
         if (!C::Bwd) { wrow = static_cast<int64_t>(mb) * 128 + row_f; kb = kt; }
         else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(mb) * 2 + c_mn; }
-        valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
+        valid = (wrow < p.w_rows[0]) && (kb < p.w_kblocks);
         return wrow * p.w_kblocks + kb;
       };
       // scale prefetch: two K steps ahead
@@ -490,8 +495,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         bool v0, v1;
         const int64_t b0 = block_of(0, v0);
         const int64_t b1 = block_of(1, v1);
-        if (0 < nmain && v0) r0 = load_raw_scale(p.scales, b0);
-        if (1 < nmain && v1) r1 = load_raw_scale(p.scales, b1);
+        if (0 < nmain && v0) r0 = load_raw_scale(p.scales[0], b0);
+        if (1 < nmain && v1) r1 = load_raw_scale(p.scales[0], b1);
       }
       for (int i = 0; i < nmain + next; ++i) {
         if (i < nmain) {
@@ -499,12 +504,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           block_of(i, valid);
           const int64_t b2 = block_of(i + 2, v2);
           RawScale r2{0u, 0.f};
-          if (i + 2 < nmain && v2) r2 = load_raw_scale(p.scales, b2);
+          if (i + 2 < nmain && v2) r2 = load_raw_scale(p.scales[0], b2);
           if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
           const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
           if (valid) {
             const uint4 w = ld_shared_v4_w(smem_u32(sR + stage * C::kRBytes) + r_off);
-            const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales, r0, mean));
+            const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales[0], r0, mean));
             const int j0 = 4 * h;
             st_shared_v4_w(adst + (((j0 + 0) ^ sw) << 4), nf4_lookup8(lut, w.x));
             st_shared_v4_w(adst + (((j0 + 1) ^ sw) << 4), nf4_lookup8(lut, w.y));
@@ -647,10 +652,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
-      tma_prefetch_desc(&maps.act);
-      tma_prefetch_desc(&maps.codes);
-      tma_prefetch_desc(&maps.a2);
-      tma_prefetch_desc(&maps.b2);
+      const int ng = (p.groups > 1) ? p.groups : 1;
+      for (int l = 0; l < ng; ++l) {
+        tma_prefetch_desc(&maps.act[l]);
+        tma_prefetch_desc(&maps.codes[l]);
+        tma_prefetch_desc(&maps.a2[l]);
+        tma_prefetch_desc(&maps.b2[l]);
+      }
       int stage = 0;
       uint32_t ph = 0;
       uint32_t pend_codes = 0, pend_full = 0, pend_par = 0;
@@ -668,39 +676,41 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           uint8_t* a_dst = sA + stage * C::kATile;
           uint8_t* b_dst = sB + stage * C::kBStage;
           if (i < nmain) {
-            const int kt = kt0 + i;
+            const int l = wlayer(p, kt0 + i);
+            const int kt = kt0 + i - p.k_begin[l];          // K step within layer l
             mbar_arrive_expect_tx(&codes_full[stage], C::kRBytes);
             if (C::Bwd) {
               if (tma_start_ok(mh * 64, kt * 64, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 20))
-                tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], mh * 64, kt * 64);
+                tma_load_2d(sR + stage * C::kRBytes, &maps.codes[l], &codes_full[stage], mh * 64, kt * 64);
             } else if (tma_start_ok(kt * 32, mh * 128, 1, p.w_kblocks * 32, sR + stage * C::kRBytes, 21)) {
-              tma_load_2d(sR + stage * C::kRBytes, &maps.codes, &codes_full[stage], kt * 32, mh * 128);
+              tma_load_2d(sR + stage * C::kRBytes, &maps.codes[l], &codes_full[stage], kt * 32, mh * 128);
             }
             pend_codes |= (1u << stage);
             if (even) mbar_arrive_expect_tx(&tma_full[stage], 2 * C::kBStage);
 #pragma unroll
             for (int t = 0; t < C::NT; ++t)
-              if (tma_start_ok(kt * 64, tok0 + t * C::BN, 2, C::Bwd ? p.w_rows : p.w_kblocks * 64,
+              if (tma_start_ok(kt * 64, tok0 + t * C::BN, 2, C::Bwd ? p.w_rows[l] : p.w_kblocks * 64,
                                b_dst + t * C::kBTile, 22))
-                tma_load_2d_pair(b_dst + t * C::kBTile, &maps.act, full_e, kt * 64, tok0 + t * C::BN);
+                tma_load_2d_pair(b_dst + t * C::kBTile, &maps.act[l], full_e, kt * 64, tok0 + t * C::BN);
           } else {
-            const int e = i - nmain;
+            const int l = (i - nmain) / p.ext_tiles;       // layer of this extension step
+            const int e = i - nmain - l * p.ext_tiles;
             // no codes for an extension step: complete codes_full's phase anyway, so that its
             // phases count every use of the stage as the dequantizers' ring phase does
             mbar_arrive(&codes_full[stage]);
             if (even) mbar_arrive_expect_tx(&tma_full[stage], 2 * (C::kATile + C::kBStage));
             if (C::Bwd) {
               if (tma_start_ok(mh * 128, e * 64, 2, p.w_kblocks * 64, a_dst, 23))
-                tma_load_2d_pair(a_dst, &maps.a2, full_e, mh * 128, e * 64);
+                tma_load_2d_pair(a_dst, &maps.a2[l], full_e, mh * 128, e * 64);
               if (tma_start_ok(mh * 128 + 64, e * 64, 2, p.w_kblocks * 64, a_dst + 8192, 24))
-                tma_load_2d_pair(a_dst + 8192, &maps.a2, full_e, mh * 128 + 64, e * 64);
+                tma_load_2d_pair(a_dst + 8192, &maps.a2[l], full_e, mh * 128 + 64, e * 64);
             } else if (tma_start_ok(e * 64, mh * 128, 2, p.ext_tiles * 64, a_dst, 25)) {
-              tma_load_2d_pair(a_dst, &maps.a2, full_e, e * 64, mh * 128);
+              tma_load_2d_pair(a_dst, &maps.a2[l], full_e, e * 64, mh * 128);
             }
 #pragma unroll
             for (int t = 0; t < C::NT; ++t)
               if (tma_start_ok(e * 64, tok0 + t * C::BN, 2, p.ext_tiles * 64, b_dst + t * C::kBTile, 26))
-                tma_load_2d_pair(b_dst + t * C::kBTile, &maps.b2, full_e, e * 64, tok0 + t * C::BN);
+                tma_load_2d_pair(b_dst + t * C::kBTile, &maps.b2[l], full_e, e * 64, tok0 + t * C::BN);
           }
           pend_full |= (1u << stage);
           pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
@@ -799,7 +809,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // main K steps in turn; each warp reports its finished tile to the even CTA's deq_full.
     const int grp = (warp - C::kDeqWarp0) >> 2;
     const int gt = threadIdx.x - 32 * C::kDeqWarp0 - 128 * grp;    // 0..127
-    const float mean = (p.scales.dq_mean != nullptr) ? __ldg(p.scales.dq_mean) : 0.f;
+    // each layer's double-quant mean (a grouped GEMM has up to kWGroupMax weights)
+    const int ng = (p.groups > 1) ? p.groups : 1;
+    const float mean0 = (p.scales[0].dq_mean != nullptr) ? __ldg(p.scales[0].dq_mean) : 0.f;
+    const float mean1 = (ng > 1 && p.scales[1].dq_mean != nullptr) ? __ldg(p.scales[1].dq_mean) : 0.f;
+    const float mean2 = (ng > 2 && p.scales[2].dq_mean != nullptr) ? __ldg(p.scales[2].dq_mean) : 0.f;
     const int i_mn = gt & 63;
     const int c_mn = gt >> 6;
     uint32_t r_off0, r_off1, a_off;
@@ -827,41 +841,46 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       const int mh = 2 * mb + rank;
       const int first = (grp - dstage % C::Groups + C::Groups) % C::Groups;   // first own main step
       constexpr int G = C::Groups;
-      auto block_of = [&](int i, bool& valid) -> int64_t {
-        const int kt = kt0 + i;
+      // block index of main step i in its layer's scales (layer returned in l)
+      auto block_of = [&](int i, bool& valid, int& l) -> int64_t {
+        l = wlayer(p, kt0 + i);
+        const int kt = kt0 + i - p.k_begin[l];
         int64_t wrow, kb;
         if (!C::Bwd) { wrow = static_cast<int64_t>(mh) * 128 + gt; kb = kt; }
         else { wrow = static_cast<int64_t>(kt) * 64 + i_mn; kb = static_cast<int64_t>(mh) * 2 + c_mn; }
-        valid = (wrow < p.w_rows) && (kb < p.w_kblocks);
+        valid = (wrow < p.w_rows[l]) && (kb < p.w_kblocks);
         return wrow * p.w_kblocks + kb;
       };
       RawScale r0{0u, 0.f}, r1{0u, 0.f}, r2{0u, 0.f}, r3{0u, 0.f};
       {
         bool v;
-        int64_t bb = block_of(first, v);
-        if (first < nmain && v) r0 = load_raw_scale(p.scales, bb);
-        bb = block_of(first + G, v);
-        if (first + G < nmain && v) r1 = load_raw_scale(p.scales, bb);
-        bb = block_of(first + 2 * G, v);
-        if (first + 2 * G < nmain && v) r2 = load_raw_scale(p.scales, bb);
-        bb = block_of(first + 3 * G, v);
-        if (first + 3 * G < nmain && v) r3 = load_raw_scale(p.scales, bb);
+        int l;
+        int64_t bb = block_of(first, v, l);
+        if (first < nmain && v) r0 = load_raw_scale(p.scales[l], bb);
+        bb = block_of(first + G, v, l);
+        if (first + G < nmain && v) r1 = load_raw_scale(p.scales[l], bb);
+        bb = block_of(first + 2 * G, v, l);
+        if (first + 2 * G < nmain && v) r2 = load_raw_scale(p.scales[l], bb);
+        bb = block_of(first + 3 * G, v, l);
+        if (first + 3 * G < nmain && v) r3 = load_raw_scale(p.scales[l], bb);
       }
       for (int i = 0; i < nmain + next; ++i) {
         if (i < nmain) {
           if (dstage % G == grp) {
             bool valid, v4;
-            block_of(i, valid);
-            const int64_t b4 = block_of(i + 4 * G, v4);
+            int l, l4;
+            block_of(i, valid, l);
+            const int64_t b4 = block_of(i + 4 * G, v4, l4);
             RawScale r4{0u, 0.f};
-            if (i + 4 * G < nmain && v4) r4 = load_raw_scale(p.scales, b4);
+            if (i + 4 * G < nmain && v4) r4 = load_raw_scale(p.scales[l4], b4);
             if (!mbar_wait(&codes_full[stage], ph)) { ok = false; break; }
             const uint32_t adst = smem_u32(sA + stage * C::kATile) + a_off;
             if (valid) {
               const uint32_t rsrc = smem_u32(sR + stage * C::kRBytes);
               const uint4 w0 = ld_shared_v4_w(rsrc + r_off0);
               const uint4 w1 = ld_shared_v4_w(rsrc + r_off1);
-              const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales, r0, mean));
+              const float mean = (l == 0) ? mean0 : (l == 1) ? mean1 : mean2;
+              const Nf4Lut lut = nf4_build_lut(p.tab, raw_to_scale(p.scales[l], r0, mean));
               st_shared_v4_w(adst + ((0 ^ sw) << 4), nf4_lookup8(lut, w0.x));
               st_shared_v4_w(adst + ((1 ^ sw) << 4), nf4_lookup8(lut, w0.y));
               st_shared_v4_w(adst + ((2 ^ sw) << 4), nf4_lookup8(lut, w0.z));

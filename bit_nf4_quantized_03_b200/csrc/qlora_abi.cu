@@ -315,6 +315,8 @@ GemmParams base_params(int64_t rows, int64_t cols, int bn, int64_t k_tiles, Spli
   // one split covers the whole reduction
   p.splits = sp.splits > 1 ? sp.splits : 1;
   p.k_per_split = sp.splits > 1 ? sp.kps : static_cast<int32_t>(k_tiles);
+  p.groups = 1;
+  for (int l = 1; l <= kWGroupMax; ++l) p.k_begin[l] = static_cast<int32_t>(k_tiles);
   p.tab = table();
   return p;
 }
@@ -432,6 +434,99 @@ int run_lora_grad(const Plan& P, const Split& sp, const uint16_t* act, int64_t m
   e = launch_grad_finalize(static_cast<const float*>(p.out), sp.splits, p.part_stride, rows, r, P.r_pad, scale, out,
                            transpose, accumulate, st);
   return cuda_status(e);
+}
+
+// One layer's share of a dX GEMM.
+struct DxLayer {
+  const qlora_nf4_weight* w;
+  const uint16_t* dY;       // [m, n_l]
+  const uint16_t* A;        // A_l [r, k]
+  const uint16_t* sG;       // bf16(s G_l) [m, r_pad]
+};
+
+// dX^T = sum_l (W_l^T . dY_l^T + A_l^T . (s G_l)^T), each W_l dequantized into the MN-major
+// operand layout: one weight GEMM whose reduction runs over the layers in turn (layers that
+// share the input X; the CTA-pair kernel alone takes more than one). `ext`: the low-rank
+// terms ride as extension K steps. Split K, and an accumulating dX on the CTA-pair path, go
+// through fp32 partials and the reduce pass: in the GEMM's epilogue the old dX values (rows
+// ld apart) were read at a small fraction of the memory's speed and stalled the tensor cores.
+int run_dx(const Plan& P, const DxLayer* L, int count, int64_t m, int64_t k, int32_t r, bool ext, void* dX,
+           int32_t dx_dtype, bool acc_dx, char* wsb, cudaStream_t st) {
+  const int bn = P.bn;
+  if (count < 1 || count > kWGroupMax || (count > 1 && wgemm_tile_rows(bn) != 256)) return QLORA_ERR_INVALID;
+  const Split& sp = P.bwd;
+  const bool via_part = sp.splits > 1 || (acc_dx && wgemm_tile_rows(bn) == 256);
+  int64_t k_tiles = 0;
+  int32_t k_begin[kWGroupMax + 1] = {};
+  for (int l = 0; l < count; ++l) {
+    k_begin[l] = static_cast<int32_t>(k_tiles);
+    k_tiles += cdiv(L[l].w->n, 64);
+  }
+  GemmParams p = base_params(k, m, bn, k_tiles, sp);
+  p.tiles_m = static_cast<int32_t>(cdiv(k, wgemm_tile_rows(bn)));
+  p.ext_tiles = ext ? P.r_pad / 64 : 0;
+  p.groups = count;
+  for (int l = 0; l <= kWGroupMax; ++l) p.k_begin[l] = (l < count) ? k_begin[l] : static_cast<int32_t>(k_tiles);
+  p.w_kblocks = k / 64;
+  for (int l = 0; l < count; ++l) {
+    p.scales[l] = scale_src(L[l].w);
+    p.w_rows[l] = static_cast<int32_t>(L[l].w->n);
+  }
+  p.ld_out = k;
+  if (via_part) {
+    p.out = wsb + P.off_part;
+    p.part_stride = m * k;
+    p.out_mode = kOutPartial;
+  } else {
+    p.out = dX;
+    p.out_mode = (dx_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
+    p.accumulate = acc_dx ? 1 : 0;
+  }
+  WMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  bool ok = true;
+  double flops = 0.0;
+  for (int l = 0; l < count; ++l) {
+    const int64_t n = L[l].w->n;
+    ok = ok && map_bf16(&maps.act[l], L[l].dY, m, n, static_cast<uint32_t>(wgemm_box_rows(bn)));
+    ok = ok && tmap_2d(&maps.codes[l], L[l].w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+                       static_cast<uint64_t>(k / 2), 64, 64, 64);
+    ok = ok && tmap_2d(&maps.a2[l], L[l].A, kBF16, k, r, k * 2, 64, 64, 128);
+    ok = ok && map_bf16(&maps.b2[l], L[l].sG, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(bn)));
+    flops += 2.0 * double(m) * double(k) * double(n + (ext ? r : 0));
+  }
+  if (!ok) return QLORA_ERR_CUDA;
+  if (launch_wgemm(true, bn, p, maps, wgemm_grid(p, bn, num_sms()), st, flops) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (via_part &&
+      launch_splitk_reduce(static_cast<const float*>(p.out), p.splits, p.part_stride, m, k, k, dX,
+                           dx_dtype == QLORA_DTYPE_BF16, acc_dx ? 1 : 0, st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
+// Workspace of a grouped backward: every layer's bf16(s G_l) (read together by the fused dX
+// GEMM), then one scratch area that the layers use in turn and the dX GEMM after them.
+struct GroupPlan {
+  size_t off_sg[kWGroupMax] = {};
+  size_t off_scratch = 0, total = 0;
+};
+
+GroupPlan make_group_plan(int32_t count, int64_t m, const int64_t* n, int64_t k, int32_t r) {
+  GroupPlan G;
+  const int r_pad = (r <= 64) ? 64 : 128;
+  size_t off = 0;
+  int64_t n_total = 0;
+  size_t scratch = 0;
+  for (int l = 0; l < count; ++l) {
+    G.off_sg[l] = off;
+    off += align_up(static_cast<size_t>(m) * r_pad * 2, 256);
+    n_total += n[l];
+    scratch = std::max(scratch, make_plan(m, n[l], k, r).total);
+  }
+  scratch = std::max(scratch, make_plan(m, n_total, k, r).total);
+  G.off_scratch = off;
+  G.total = off + scratch;
+  return G;
 }
 
 }  // namespace
@@ -579,9 +674,9 @@ int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m,
   GemmParams p = base_params(n, m, P.bn, k / 64, P.fwd);
   p.tiles_m = static_cast<int32_t>(cdiv(n, wgemm_tile_rows(P.bn)));
   p.ext_tiles = P.r_pad / 64;
-  p.scales = scale_src(w);
+  p.scales[0] = scale_src(w);
   p.w_kblocks = k / 64;
-  p.w_rows = static_cast<int32_t>(n);
+  p.w_rows[0] = static_cast<int32_t>(n);
   p.ld_out = n;
   if (P.fwd.splits > 1) {
     p.out = wsb + P.off_part;
@@ -593,11 +688,11 @@ int qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t m,
   }
   WMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  bool ok = map_bf16(&maps.act, X, m, k, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
-  ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
+  bool ok = map_bf16(&maps.act[0], X, m, k, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
+  ok = ok && tmap_2d(&maps.codes[0], w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
                      static_cast<uint64_t>(k / 2), 32, 128, 32);
-  ok = ok && tmap_2d(&maps.a2, B, kBF16, r, n, r * 2, 64, 128, 128);
-  ok = ok && map_bf16(&maps.b2, sU, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
+  ok = ok && tmap_2d(&maps.a2[0], B, kBF16, r, n, r * 2, 64, 128, 128);
+  ok = ok && map_bf16(&maps.b2[0], sU, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(P.bn)));
   if (!ok) return QLORA_ERR_CUDA;
   const double fwd_flops = 2.0 * double(m) * double(n) * double(k + r);
   // at few tokens U comes from lora_down_small_kernel right before: the GEMM may start streaming
@@ -666,45 +761,9 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
   }
 
   if (dX != nullptr) {
-    // dX^T = W^T . dY^T + A^T . (sG)^T, W dequantized into the MN-major operand layout
-    const int acc_dx = (flags & QLORA_BWD_ACCUMULATE_DX) ? 1 : 0;
-    const int bn = P.bn;
-    const Split& sp = P.bwd;
-    // Accumulating on the CTA-pair path goes through fp32 partials and the reduce pass: in the
-    // GEMM's epilogue the old dX values (rows ld apart) were read at a small fraction of the
-    // memory's speed and stalled the tensor cores; the streaming reduce reads them coalesced.
-    const bool via_part = sp.splits > 1 || (acc_dx && wgemm_tile_rows(bn) == 256);
-    GemmParams p = base_params(k, m, bn, cdiv(n, 64), sp);
-    p.tiles_m = static_cast<int32_t>(cdiv(k, wgemm_tile_rows(bn)));
-    p.ext_tiles = D.on ? 0 : P.r_pad / 64;     // under dropout the low-rank term is added masked, below
-    p.scales = scale_src(w);
-    p.w_kblocks = k / 64;
-    p.w_rows = static_cast<int32_t>(n);
-    p.ld_out = k;
-    if (via_part) {
-      p.out = wsb + P.off_part;
-      p.part_stride = m * k;
-      p.out_mode = kOutPartial;
-    } else {
-      p.out = dX;
-      p.out_mode = (dx_dtype == QLORA_DTYPE_FP32) ? kOutF32 : kOutBF16;
-      p.accumulate = acc_dx;
-    }
-    WMaps maps;
-    std::memset(&maps, 0, sizeof(maps));
-    bool ok = map_bf16(&maps.act, dY, m, n, static_cast<uint32_t>(wgemm_box_rows(bn)));
-    ok = ok && tmap_2d(&maps.codes, w->codes, kU8, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n),
-                       static_cast<uint64_t>(k / 2), 64, 64, 64);
-    ok = ok && tmap_2d(&maps.a2, A, kBF16, k, r, k * 2, 64, 64, 128);
-    ok = ok && map_bf16(&maps.b2, sG, m, P.r_pad, static_cast<uint32_t>(wgemm_box_rows(bn)));
-    if (!ok) return QLORA_ERR_CUDA;
-    const double dx_flops = 2.0 * double(m) * double(k) * double(n + r);
-    if (launch_wgemm(true, bn, p, maps, wgemm_grid(p, bn, num_sms()), st, dx_flops) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    if (via_part &&
-        launch_splitk_reduce(static_cast<const float*>(p.out), p.splits, p.part_stride, m, k, k, dX,
-                             dx_dtype == QLORA_DTYPE_BF16, acc_dx, st) != cudaSuccess)
-      return QLORA_ERR_CUDA;
+    const DxLayer L{w, dY, A, sG};
+    rc = run_dx(P, &L, 1, m, k, r, !D.on, dX, dx_dtype, (flags & QLORA_BWD_ACCUMULATE_DX) != 0, wsb, st);
+    if (rc != QLORA_OK) return rc;
     if (D.on) {
       rc = run_lora_up_masked(P, sG, m, k, A, r, D, dX, dx_dtype == QLORA_DTYPE_FP32, st);
       if (rc != QLORA_OK) return rc;
@@ -715,6 +774,89 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
   if (rc != QLORA_OK) return rc;
   rc = run_lora_grad(P, P.da, Xl, m, k, g_hi, g_lo, r, D.on ? s * D.keep : s, dA, 1, acc_grads, wsb, st);
   return rc;
+}
+
+size_t qlora_linear_group_workspace_bytes(int32_t count, int64_t m, const int64_t* n, int64_t k, int32_t r) {
+  if (count < 1 || count > kWGroupMax || n == nullptr || m < 1 || k < 1 || r < 1 || r > 128) return 0;
+  for (int l = 0; l < count; ++l)
+    if (n[l] < 1) return 0;
+  return make_group_plan(count, m, n, k, r).total;
+}
+
+int qlora_linear_bwd_group(int32_t count, const qlora_nf4_weight* const* w, const uint16_t* X,
+                           const uint16_t* const* dY, int64_t m, const uint16_t* const* A, const uint16_t* const* B,
+                           int32_t r, float alpha, const float* const* U_saved, void* dX, int32_t dx_dtype,
+                           float* const* dA, float* const* dB, int32_t flags, void* ws, size_t ws_bytes,
+                           qlora_stream_t stream) {
+  if (count < 1 || count > kWGroupMax || w == nullptr || dY == nullptr || A == nullptr || B == nullptr ||
+      dA == nullptr || dB == nullptr)
+    return QLORA_ERR_INVALID;
+  if ((flags & ~(QLORA_BWD_ACCUMULATE_GRADS | QLORA_BWD_ACCUMULATE_DX)) != 0) return QLORA_ERR_INVALID;
+  if (dX != nullptr && (!aligned16(dX) || (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_FP32)))
+    return QLORA_ERR_INVALID;
+  int64_t n[kWGroupMax] = {};
+  for (int l = 0; l < count; ++l) {
+    if (!linear_args_ok(w[l], X, m, A[l], B[l]) || dY[l] == nullptr || !aligned16(dY[l])) return QLORA_ERR_INVALID;
+    if (dA[l] == nullptr || dB[l] == nullptr || !aligned16(dA[l]) || !aligned16(dB[l])) return QLORA_ERR_INVALID;
+    if (U_saved != nullptr && U_saved[l] != nullptr && !aligned16(U_saved[l])) return QLORA_ERR_INVALID;
+    if (w[l]->k != w[0]->k) return QLORA_ERR_INVALID;
+    const int sst = linear_shape_status(w[l], r);
+    if (sst != QLORA_OK) return sst;
+    n[l] = w[l]->n;
+  }
+  const int64_t k = w[0]->k;
+  const GroupPlan G = make_group_plan(count, m, n, k, r);
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < G.total) return QLORA_ERR_WORKSPACE;
+  char* wsb = static_cast<char*>(ws);
+  char* scratch = wsb + G.off_scratch;
+  const size_t scratch_bytes = G.total - G.off_scratch;
+  int64_t n_total = 0;
+  for (int l = 0; l < count; ++l) n_total += n[l];
+  const Plan Pg = make_plan(m, n_total, k, r);
+  const int acc_dx = flags & QLORA_BWD_ACCUMULATE_DX;
+  const int acc_grads = flags & QLORA_BWD_ACCUMULATE_GRADS;
+
+  if (count == 1 || dX == nullptr || wgemm_tile_rows(Pg.bn) != 256) {
+    // one layer, no dX, or few tokens (the single-CTA weight GEMM takes one layer): the layers
+    // one after the other, each adding its dX term to the previous ones
+    for (int l = 0; l < count; ++l) {
+      const int32_t fl = acc_grads | ((l > 0 || acc_dx) ? QLORA_BWD_ACCUMULATE_DX : 0);
+      const int rc = qlora_linear_bwd_ex(w[l], X, dY[l], m, A[l], B[l], r, alpha,
+                                         U_saved != nullptr ? U_saved[l] : nullptr, dX, dx_dtype, dA[l], dB[l], fl,
+                                         nullptr, scratch, scratch_bytes, stream);
+      if (rc != QLORA_OK) return rc;
+    }
+    return QLORA_OK;
+  }
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float s = alpha / static_cast<float>(r);
+  DxLayer L[kWGroupMax];
+  for (int l = 0; l < count; ++l) {
+    // G_l = dY_l B_l: bf16(s G_l) kept for the dX GEMM, hi/lo bf16 for dA_l; the saved U_l's
+    // hi/lo split for dB_l in the same finalize launch (or U_l recomputed)
+    const Plan P = make_plan(m, n[l], k, r);
+    uint16_t* sG = reinterpret_cast<uint16_t*>(wsb + G.off_sg[l]);
+    uint16_t* g_hi = reinterpret_cast<uint16_t*>(scratch + P.off_hi_b);
+    uint16_t* g_lo = reinterpret_cast<uint16_t*>(scratch + P.off_lo_b);
+    uint16_t* u_hi = reinterpret_cast<uint16_t*>(scratch + P.off_hi_a);
+    uint16_t* u_lo = reinterpret_cast<uint16_t*>(scratch + P.off_lo_a);
+    const float* Us = (U_saved != nullptr) ? U_saved[l] : nullptr;
+    int rc = run_lora_down(P, true, dY[l], m, n[l], B[l], r, s, scratch, nullptr, sG, g_hi, g_lo, st, 1.0f, Us,
+                           Us != nullptr ? u_hi : nullptr, Us != nullptr ? u_lo : nullptr);
+    if (rc != QLORA_OK) return rc;
+    if (Us == nullptr) {
+      rc = run_lora_down(P, false, X, m, k, A[l], r, s, scratch, nullptr, nullptr, u_hi, u_lo, st);
+      if (rc != QLORA_OK) return rc;
+    }
+    rc = run_lora_grad(P, P.db, dY[l], m, n[l], u_hi, u_lo, r, s, dB[l], 0, acc_grads, scratch, st);
+    if (rc != QLORA_OK) return rc;
+    rc = run_lora_grad(P, P.da, X, m, k, g_hi, g_lo, r, s, dA[l], 1, acc_grads, scratch, st);
+    if (rc != QLORA_OK) return rc;
+    L[l] = DxLayer{w[l], dY[l], A[l], sG};
+  }
+  // dX = sum_l (dY_l W_l + s G_l A_l): one weight GEMM over the layers' reductions in turn
+  return run_dx(Pg, L, count, m, k, r, true, dX, dx_dtype, acc_dx != 0, scratch, st);
 }
 
 int qlora_adamw_step(float* param, const float* grad, float* m, float* v, uint16_t* param_bf16, int64_t count,

@@ -63,16 +63,25 @@ enum OutMode : int {
   kOutMaskAccF32 = 4,   // fp32 out, same
 };
 
+// Layers at most in one grouped weight GEMM (the backward of projections that share an
+// input: q, k and v; or gate and up).
+constexpr int kWGroupMax = 3;
+
 struct GemmParams {
   int32_t rows, cols;          // problem size of D
   int32_t tiles_m, tiles_n;    // 128-row and BN-col tiles
   int32_t k_tiles;             // main-loop 64-wide K steps
   int32_t ext_tiles;           // extra K steps from the second operand pair (low-rank branch)
   int32_t splits, k_per_split; // split of the main K steps
-  // NF4 operand (weight-operand GEMM only)
-  ScaleSrc scales;
-  int64_t w_kblocks;           // 64-blocks per row of W
-  int32_t w_rows;              // rows of W
+  // NF4 operand (weight-operand GEMM only). A grouped GEMM (CTA-pair kernel, backward)
+  // runs its reduction over the layers in turn: layer l owns main K steps
+  // [k_begin[l], k_begin[l + 1]) and extension steps [l * ext_tiles, (l + 1) * ext_tiles)
+  // after every main step; one layer: groups = 1, k_begin = {0, k_tiles}.
+  int32_t groups;
+  int32_t k_begin[kWGroupMax + 1];
+  ScaleSrc scales[kWGroupMax];
+  int64_t w_kblocks;           // 64-blocks per row of W (the same for every layer of a group)
+  int32_t w_rows[kWGroupMax];  // rows of each layer's W
   // output
   void* out;
   int64_t ld_out;
@@ -153,11 +162,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, siz
 // 128-row MMA operand. GemmParams: rows = features (n forward, k backward),
 // cols = tokens, tiles_m = features / 128, tiles_n = tokens / BN; the output is
 // row-major [tokens, ld_out] (Y or dX), split partials the same way.
-struct WMaps {
-  CUtensorMap act;     // activations [tokens, reduction] bf16, box [64, BN], 128B swizzle
-  CUtensorMap codes;   // packed codes [n, k/2] u8; forward box [32, 128] (32B swizzle), backward [64, 64] (64B)
-  CUtensorMap a2;      // low-rank A-side tile: B_lora [n, r] (forward) or A_lora [r, k] (backward)
-  CUtensorMap b2;      // low-rank B-side tile: s*U or s*G [tokens, r_pad]
+struct WMaps {          // one entry per layer of a group ([0] alone for one layer)
+  CUtensorMap act[kWGroupMax];     // activations [tokens, reduction] bf16, box [64, BN], 128B swizzle
+  CUtensorMap codes[kWGroupMax];   // packed codes [n, k/2] u8; forward box [32, 128] (32B swizzle), backward [64, 64] (64B)
+  CUtensorMap a2[kWGroupMax];      // low-rank A-side tile: B_lora [n, r] (forward) or A_lora [r, k] (backward)
+  CUtensorMap b2[kWGroupMax];      // low-rank B-side tile: s*U or s*G [tokens, r_pad]
 };
 int wgemm_bn(int64_t tokens);          // tokens per tile
 int wgemm_box_rows(int bn);              // token rows per TMA box (each CTA of a pair loads half)

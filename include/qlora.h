@@ -273,6 +273,43 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight *w, const uint16_t *X, const uint
                         const qlora_dropout *drop, void *ws, size_t ws_bytes, qlora_stream_t stream);
 
 /*
+ * Backward of up to three layers that read the same input X: the q, k and v
+ * projections of an attention block, or the gate and up projections of a SiLU
+ * MLP (the pages put LoRA on every linear layer: "QLoRA Explained", Step 3,
+ * target_modules = "all-linear"). For layer l = 0 .. count - 1, with weight
+ * w[l] ([n_l, k]; k the same for all), dY[l] [m, n_l], adapters A[l] [r, k]
+ * and B[l] [n_l, r], and the same r and alpha:
+ *   dX[m, k] (+)= sum_l (dY_l W'_l + (alpha/r) (dY_l B_l) A_l)
+ *   dA[l], dB[l] (+)= as qlora_linear_bwd gives them for layer l
+ * The value is that of qlora_linear_bwd called per layer with
+ * QLORA_BWD_ACCUMULATE_DX from the second layer on; the sum is formed in one
+ * fused GEMM whose reduction runs over the layers in turn (above 128 tokens),
+ * so no layer's term passes through an fp32 partial. At most 128 tokens, or
+ * with dX NULL, the layers run one after the other.
+ *  - w, dY, A, B, dA, dB: arrays of count pointers, each as in
+ *    qlora_linear_bwd; U_saved: NULL or an array of count pointers, each NULL
+ *    (U_l recomputed) or fp32 [m, r] from that layer's forward.
+ *  - flags: QLORA_BWD_ACCUMULATE_GRADS (every layer's dA, dB) and/or
+ *    QLORA_BWD_ACCUMULATE_DX.
+ *  - No LoRA dropout here (qlora_linear_bwd_ex per layer has it).
+ *  - ws: qlora_linear_group_workspace_bytes(count, m, n, k, r) bytes, 16-byte
+ *    aligned, device memory; the call reads and writes it and nothing else
+ *    keeps it.
+ *  - count outside 1..3, differing k, or an argument qlora_linear_bwd would
+ *    reject: the same status as there, with nothing enqueued.
+ */
+int qlora_linear_bwd_group(int32_t count, const qlora_nf4_weight *const *w, const uint16_t *X,
+                           const uint16_t *const *dY, int64_t m, const uint16_t *const *A,
+                           const uint16_t *const *B, int32_t r, float alpha, const float *const *U_saved,
+                           void *dX, int32_t dx_dtype, float *const *dA, float *const *dB, int32_t flags,
+                           void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Workspace of qlora_linear_bwd_group for count layers with n[l] output
+ * features each (array of count), k input features, m tokens and rank r;
+ * 0 for arguments it would reject. */
+size_t qlora_linear_group_workspace_bytes(int32_t count, int64_t m, const int64_t *n, int64_t k, int32_t r);
+
+/*
  * Paged AdamW, 32-bit, for the adapters ("QLoRA Explained": Paged Optimizers
  * and optim = "paged_adamw_32bit"; "QLoRA: Quantized Low-Rank Adaptation":
  * "Paged optimizers (the storage unit)"). AdamW with decoupled weight decay

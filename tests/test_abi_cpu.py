@@ -165,3 +165,13 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(TypeError):
         q._ptr(1 << 20)
     assert q._ptr(1 << 20, allow_addr=True) == 1 << 20
+
+
+def test_binding_constants_match_the_header_enums():
+    # every QLORA_* enum value the header defines, as the binding spells it
+    import re
+    text = open(HEADER).read()
+    vals = dict((name, int(v)) for name, v in re.findall(r"\b(QLORA_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    assert vals, "no enum values found"
+    for name, v in vals.items():
+        assert getattr(q, name) == v, name
