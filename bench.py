@@ -46,12 +46,12 @@ LAYERS = [("q_proj", 8192, 8192), ("k_proj", 8192, 8192), ("v_proj", 8192, 8192)
 L2_FLUSH_BYTES = 512 << 20
 PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12) flops, one at 16 tokens <= 5.8e9
 
-# DRAM bytes (read + write) per launch of the CTA-pair fused GEMM, averaged over its 14 launches of one step, from the
+# DRAM bytes (read + write) per launch of the CTA-pair fused GEMM, averaged over its 11 launches of one step, from the
 # 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum). Printed only while the
 # kernel's sources hash to the value recorded with it; any change to them prints null until the counters are taken
 # again.
-WGEMM_TRAFFIC = {"bytes_per_launch": 920445495,
-                 "sources_sha256": "3959e96c205beb70922c1f9ff599d89536741d9f65ddc973e784c89b05be6ea5"}
+WGEMM_TRAFFIC = {"bytes_per_launch": 1212925451,
+                 "sources_sha256": "add11e86b6cdf55f3cdd68377db3696e58dfdae5bf7a54e725c2753d0b6c968d"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 
@@ -61,6 +61,25 @@ def wgemm_sources_sha256() -> str:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
+
+
+def pair_algo_bytes(m: int = M_TOKENS, r: int = RANK_R) -> float:
+    """Algorithmic DRAM bytes per CTA-pair launch of one step, averaged over its launches:
+    every operand counted once at its stored size (bf16 activations and outputs, packed
+    codes, E4M3 scales with their fp32 second-level scales, the adapter tiles of the K
+    extension). Forward: X, W, Y per layer; backward: the layers of a group (q/k/v, and
+    gate/up) in one launch reading every layer's dY and W and writing dX once."""
+    def w_bytes(n, k):
+        return n * k * (0.5 + 1.0 / 64 + 4.0 / 16384)
+    dims = {nm: (n, k) for nm, n, k in LAYERS}
+    launches = []
+    for nm, n, k in LAYERS:                                        # forwards
+        launches.append(2 * m * k + w_bytes(n, k) + 2 * m * n + 2 * m * r + 2 * n * r)
+    for group in (("down_proj",), ("gate_proj", "up_proj"), ("o_proj",), ("q_proj", "k_proj", "v_proj")):
+        k = dims[group[0]][1]
+        launches.append(2 * m * k + sum(2 * m * dims[g][0] + w_bytes(*dims[g]) + 2 * m * r + 2 * r * k
+                                        for g in group))
+    return sum(launches) / len(launches)
 
 
 def wgemm_traffic():
@@ -677,6 +696,20 @@ def components(dev, peaks) -> dict:
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for qn, qk, sfx in ((4096, 4096, ""), (22016, 8192, "_65b_gate")):
         _quant_components(q, synth, torch, dev, flush, peaks, out, qn, qk, sfx)
+    # what a plain device copy reaches when it moves the same bytes as the 4096 x 4096
+    # quantize (76 MB) and dequantize (42 MB), timed the same way: the bandwidth a kernel of
+    # this size can see, beside the 2 GB copy the peak comes from
+    for tag in ("quantize_bf16", "dequantize_bf16"):
+        half = int(out[tag]["algo_bytes"]) // 2 // 16 * 16
+        src = torch.empty(half, dtype=torch.uint8, device=dev)
+        dst = torch.empty(half, dtype=torch.uint8, device=dev)
+        fn = lambda: dst.copy_(src)
+        for _ in range(3):
+            fn()
+        ms = graph_time(fn, 20, flush)
+        out[f"copy_same_bytes_as_{tag}"] = {"us": ms * 1e3, "gbs": 2 * half / ms / 1e6,
+                                            "frac": 2 * half / ms / 1e6 / peaks["hbm_gbs"], "bytes_moved": 2 * half}
+        del src, dst
     _seven_b_components(q, synth, torch, dev, flush, peaks, out)
     # the NF4 expansion alone on every SM: the ceiling on the weight rate of any kernel that
     # turns each weight into BF16 through the per-block table
@@ -965,7 +998,9 @@ def run_native(args) -> None:
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
                 "frac": (achieved / peak_tc) if achieved else None, "traffic": wgemm_traffic(),
-                "traffic_unit": "DRAM bytes per launch, average over the step's 14 CTA-pair launches (ncu)",
+                "traffic_unit": "DRAM bytes per launch, average over the step's 11 CTA-pair launches (ncu): seven "
+                                "forwards, four backwards (q/k/v and gate/up grouped)",
+                "algorithmic_bytes_per_launch": pair_algo_bytes(),
                 "kernel": "qlora_wgemm_pair_kernel (fused NF4 dequant + tcgen05 cta_group::2, 256 weight rows x 512 "
                           "tokens per CTA pair; forward Y and backward dX at 8192 tokens)",
                 "launches_timed": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1),

@@ -62,7 +62,8 @@ struct WCfg {
   static_assert(kGroups == 1 || (kGroups >= 2 && kStages % kGroups == 0), "the stage index modulo G picks the group");
 };
 
-constexpr int kRasterGroup = 4;   // token tiles per raster group (L2 reuse of both operands)
+// Token tiles per raster group (L2 reuse of both operands): p.raster when set, else 4.
+constexpr int kRasterGroup = 4;
 constexpr int64_t kPair512From = 1024;   // above this many tokens a CTA pair takes 512 per unit
 
 
@@ -70,13 +71,14 @@ __device__ __forceinline__ void wdecode(const GemmParams& p, int u, int& mb, int
                                         int& nmain, int& next) {
   split = u % p.splits;
   const int t = u / p.splits;
-  const int per_group = kRasterGroup * p.tiles_m;
+  const int rg = (p.raster > 0) ? p.raster : kRasterGroup;
+  const int per_group = rg * p.tiles_m;
   const int g = t / per_group;
   const int within = t - g * per_group;
-  int gsize = p.tiles_n - g * kRasterGroup;
-  if (gsize > kRasterGroup) gsize = kRasterGroup;
+  int gsize = p.tiles_n - g * rg;
+  if (gsize > rg) gsize = rg;
   mb = within / gsize;
-  nb = g * kRasterGroup + (within - mb * gsize);
+  nb = g * rg + (within - mb * gsize);
   kt0 = split * p.k_per_split;
   int kt1 = kt0 + p.k_per_split;
   if (kt1 > p.k_tiles) kt1 = p.k_tiles;

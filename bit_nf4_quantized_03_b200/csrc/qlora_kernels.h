@@ -92,6 +92,8 @@ struct GemmParams {
   // masked modes: bit (row * ld_out + col) of `mask` (bit e % 8 of byte e / 8) keeps the element
   const uint8_t* mask;
   float keep_scale;
+  // weight GEMM: token tiles per raster group (0 = the kernel's default)
+  int32_t raster;
   // single-CTA weight GEMM only (set by launch_wgemm): 1 = started before the grid that
   // writes the low-rank operand has finished; only the producer waits, before its first
   // extension load
