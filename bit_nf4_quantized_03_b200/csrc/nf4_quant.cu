@@ -33,13 +33,15 @@ __device__ int g_bounds_site = 0;
 // of its 32 weights (32 independent chains), and writes them as one 16-byte
 // store. A ragged last block is read from global memory.
 //
-// The code of x = w * (1/absmax) is found with one comparison: [-1 - 1/16,
-// 1 + 1/16) is cut into 35 buckets of width 1/16, each widened by 1e-3; the
-// widened bucket holds at most one decision threshold (neighbouring
+// The code of x = w * (1/absmax) is found with one comparison: x's bucket is
+// j = round(16 x) (-16 .. 16), the buckets [j/16 - 1/32, j/16 + 1/32] widened
+// by 1e-3; a widened bucket holds at most one decision threshold (neighbouring
 // thresholds are >= 0.08 apart), so code = (thresholds below the bucket) +
 // (x > the bucket's threshold), exactly the number of thresholds strictly
-// below x. The bucket index only has to be right up to the widening, which
-// covers the rounding of x * 16 + 16.5 and of the round-to-integer below.
+// below x. j comes out of one fused multiply-add, 1.5 * 2^23 + 16 x rounded to
+// an integer (the sum's ulp is 1), whose low six bits, inserted at bit 3 of
+// the 512-byte aligned table's address, address the 8-byte entry of j mod 64;
+// the widening covers ties and the rounding.
 //
 // In double-quant mode each chunk's 128 absmax values are also reduced in
 // fp64 with the fixed pairwise tree (the first levels of the tensor-wide sum
@@ -52,11 +54,14 @@ constexpr int kQCtasPerSm = 2;    // resident CTAs per SM (shared memory: kQStag
 constexpr int kQStage = kQChunk * 256;                // bytes per stage: two 16 KB boxes of half-blocks
 constexpr int kQSmem = kQStages * kQStage + 1024;     // + alignment of the swizzled stages
 
-__device__ __forceinline__ uint32_t nf4_code_bucket(float x, const float2* tab) {
-  // bucket = floor(x * 16 + 17): round-to-integer of x * 16 + 16.5 by adding 1.5 * 2^23
-  const float r = __fadd_rn(__fmaf_rn(x, 16.0f, 16.5f), 12582912.0f);
-  const float2 e = tab[__float_as_uint(r) & 63u];
-  return static_cast<uint32_t>(__float_as_int(e.y)) + ((x > e.x) ? 1u : 0u);
+__device__ __forceinline__ uint32_t nf4_code_bucket(float x, uint32_t tab_addr) {
+  const float r = __fmaf_rn(x, 16.0f, 12582912.0f);     // 1.5 * 2^23 + round(16 x)
+  uint32_t a;
+  asm("bfi.b32 %0, %1, %2, 3, 6;" : "=r"(a) : "r"(__float_as_uint(r)), "r"(tab_addr));
+  float thr;
+  uint32_t base;
+  asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(thr), "=r"(base) : "r"(a));
+  return base + ((x > thr) ? 1u : 0u);
 }
 
 __device__ __forceinline__ uint32_t bfi4(uint32_t word, uint32_t code, uint32_t pos) {
@@ -67,7 +72,7 @@ __device__ __forceinline__ uint32_t bfi4(uint32_t word, uint32_t code, uint32_t 
 
 // Codes of one lane's eight weights (x = w * inv); the first four (lo) go to
 // nibbles 0..3 of the 16-bit result, the next four (hi) to nibbles 4..7.
-__device__ __forceinline__ uint32_t nf4_codes8(const float4& lo, const float4& hi, float inv, const float2* tab) {
+__device__ __forceinline__ uint32_t nf4_codes8(const float4& lo, const float4& hi, float inv, uint32_t tab) {
   uint32_t w = 0;
   w = bfi4(w, nf4_code_bucket(__fmul_rn(lo.x, inv), tab), 0);
   w = bfi4(w, nf4_code_bucket(__fmul_rn(lo.y, inv), tab), 4);
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
     if (threadIdx.x == 0) atomicExch(&g_device_error, kErrBadLayout);
     return;
   }
-  __shared__ float2 s_tab[64];
+  __shared__ __align__(512) float2 s_tab[64];       // entry j mod 64 for bucket j = round(16 x)
   __shared__ double s_part[2][8];             // per chunk: the eight warps' sums of 16 blocks (by chunk parity)
   __shared__ __align__(8) uint64_t full[kQStages];
   const int tid = threadIdx.x;
@@ -159,11 +164,15 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
   const int64_t nblk = nfull + (tail > 0 ? 1 : 0);
   const int64_t nchunks = (nblk + kQChunk - 1) / kQChunk;
   const int64_t my_n = (nchunks > blockIdx.x) ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if ((smem_u32(s_tab) & 511u) != 0u) {      // the bucket address is built by inserting bits 3..8
+    if (tid == 0) atomicExch(&g_device_error, kErrBadLayout);
+    return;
+  }
   if (tid < 64) {
-    // entry b covers [(b - 1)/16 - 1, b/16 - 1); entries 35.. are never indexed
-    const int b = tid;
-    s_tab[b] = (b < 35) ? make_float2(bk.thr[b], __int_as_float(bk.base[b]))
-                        : make_float2(__int_as_float(0x7f800000), __int_as_float(15));
+    // slot t holds bucket j = t (t < 32) or t - 64; only j = -16 .. 16 are ever indexed
+    const int j = (tid < 32) ? tid : tid - 64;
+    s_tab[tid] = (j >= -16 && j <= 16) ? make_float2(bk.thr[j + 16], __int_as_float(bk.base[j + 16]))
+                                       : make_float2(__int_as_float(0x7f800000), __int_as_float(15));
   }
   if (tid == 0) {
     for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
@@ -226,10 +235,11 @@ __global__ void __launch_bounds__(256, kQCtasPerSm) nf4_quantize_kernel(const __
     uint4 word = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);  // zero or subnormal absmax
     if (cls != 2 && m >= 1.17549435e-38f) {
       const float inv = __frcp_rn(m);
-      word.x = nf4_codes8(v[0], v[1], inv, s_tab);
-      word.y = nf4_codes8(v[2], v[3], inv, s_tab);
-      word.z = nf4_codes8(v[4], v[5], inv, s_tab);
-      word.w = nf4_codes8(v[6], v[7], inv, s_tab);
+      const uint32_t tab = smem_u32(s_tab);
+      word.x = nf4_codes8(v[0], v[1], inv, tab);
+      word.y = nf4_codes8(v[2], v[3], inv, tab);
+      word.z = nf4_codes8(v[4], v[5], inv, tab);
+      word.w = nf4_codes8(v[6], v[7], inv, tab);
     }
     if (cls == 0) {
       if (qlora_check((b + 1) * 64 <= n_elem, 53)) *reinterpret_cast<uint4*>(codes + b * 32 + h * 16) = word;

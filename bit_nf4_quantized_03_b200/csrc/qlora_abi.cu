@@ -29,12 +29,13 @@ std::vector<double> g_last_ms, g_last_flops;   // per launch, from the last qlor
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 Nf4Buckets nf4_buckets_from_midpoints(const float* mid) {
-  // Widened buckets [(b-1)/16 - 1 - eps, b/16 - 1 + eps]: neighbouring thresholds are
-  // >= 0.08 apart, wider than a widened bucket, so each holds at most one.
+  // Widened buckets [j/16 - 1/32 - eps, j/16 + 1/32 + eps], j = b - 16: neighbouring
+  // thresholds are >= 0.08 apart, wider than a widened bucket, so each holds at most one.
   const double eps = 1e-3;
   Nf4Buckets bk;
-  for (int b = 0; b < 35; ++b) {
-    const double lo = (b - 1) / 16.0 - 1.0 - eps, hi = b / 16.0 - 1.0 + eps;
+  for (int b = 0; b < kNf4Buckets; ++b) {
+    const double j = b - 16;
+    const double lo = j / 16.0 - 1.0 / 32.0 - eps, hi = j / 16.0 + 1.0 / 32.0 + eps;
     int below = 0;
     float thr = INFINITY;
     for (int i = 0; i < 15; ++i) {

@@ -20,13 +20,15 @@ struct Nf4Table {
   float mid[16];
 };
 
-// Exact one-comparison code search for the quantizer: 35 buckets of width
-// 1/16, bucket b = [(b - 1)/16 - 1, b/16 - 1), each widened by 1e-3; thr[b]
-// is the single decision threshold inside widened bucket b (+inf if none)
-// and base[b] the number of thresholds below it. code(x) = base[b] + (x > thr[b]).
+// Exact one-comparison code search for the quantizer: 33 buckets of width
+// 1/16 centred on j/16, j = -16 .. 16 (entry j + 16): bucket j is the x with
+// round(16 x) = j, [j/16 - 1/32, j/16 + 1/32], widened by 1e-3 on each side;
+// thr is the single decision threshold inside the widened bucket (+inf if
+// none) and base the number of thresholds below it. code(x) = base + (x > thr).
+constexpr int kNf4Buckets = 33;
 struct Nf4Buckets {
-  float thr[35];
-  int32_t base[35];
+  float thr[kNf4Buckets];
+  int32_t base[kNf4Buckets];
 };
 
 // Device error word: kernels write a non-zero code here when a bounded wait
