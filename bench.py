@@ -51,7 +51,7 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # kernel's sources hash to the value recorded with it; any change to them prints null until the counters are taken
 # again.
 WGEMM_TRAFFIC = {"bytes_per_launch": 1212925451,
-                 "sources_sha256": "add11e86b6cdf55f3cdd68377db3696e58dfdae5bf7a54e725c2753d0b6c968d"}
+                 "sources_sha256": "a35be1bbb55c0ef1ce6e68dde5c654e77858a2b26d44fc81785bda2957fb09fe"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 
