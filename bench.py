@@ -849,6 +849,26 @@ def run_case(args) -> None:
                 q.qlora_linear_bwd(qw, x, dy, a, b, RANK_R, ALPHA, u, dx, q.QLORA_DTYPE_BF16, da, db, 0, ws)
             else:
                 q.qlora_linear_fwd(qw, x, a, b, RANK_R, ALPHA, y, q.QLORA_DTYPE_BF16, u, ws)
+    elif name == "bwd_qkv_group_65b":
+        # the grouped q/k/v backward at 8192 tokens (three 8192 x 8192 weights sharing X)
+        n, k = LAYERS[0][1], LAYERS[0][2]
+        mem = []
+        for i in range(3):
+            W = synth.weight(n, k, layer=i).to(dev)
+            qw = q.QuantizedWeight(n, k, q.QLORA_SCALE_DQ_FP8, device=dev)
+            q.qlora_nf4_quantize(W, qw)
+            del W
+            a, b = (t.to(dev) for t in synth.lora_pair(RANK_R, k, n, layer=i))
+            mem.append((qw, a, b, synth.grad_output(M_TOKENS, n, layer=20 + i).to(dev)))
+        x = synth.activations(M_TOKENS, k).to(dev)
+        dx = torch.empty(M_TOKENS, k, dtype=torch.bfloat16, device=dev)
+        grads = [(torch.empty(RANK_R, k, device=dev), torch.empty(n, RANK_R, device=dev)) for _ in mem]
+        ws = torch.empty(q.qlora_linear_group_workspace_bytes(M_TOKENS, [n] * 3, k, RANK_R), dtype=torch.uint8,
+                         device=dev)
+        for _ in range(1 + args.case_iters):
+            q.qlora_linear_bwd_group([m_[0] for m_ in mem], x, [m_[3] for m_ in mem], [m_[1] for m_ in mem],
+                                     [m_[2] for m_ in mem], RANK_R, ALPHA, None, dx, q.QLORA_DTYPE_BF16,
+                                     [g[0] for g in grads], [g[1] for g in grads], 0, ws)
     elif name == "q_proj_7b":
         # 7B q_proj fwd+bwd at 2048 tokens (4096 x 4096, r = 64)
         M, N, K = 2048, 4096, 4096
