@@ -322,9 +322,10 @@ GemmParams base_params(int64_t rows, int64_t cols, int bn, int64_t k_tiles, Spli
   return p;
 }
 
-int grid_of(const GemmParams& p) {
+// Persistent grid of a low-rank GEMM: one CTA per unit, at most one per SM, or `cap`.
+int grid_of(const GemmParams& p, int cap = 0) {
   const int64_t units = static_cast<int64_t>(p.tiles_m) * p.tiles_n * p.splits;
-  return static_cast<int>(std::min<int64_t>(units, num_sms()));
+  return static_cast<int>(std::min<int64_t>(units, cap > 0 ? cap : num_sms()));
 }
 
 const CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -418,7 +419,7 @@ int run_lora_up_masked(const Plan& P, const uint16_t* sG, int64_t m, int64_t k, 
 // dB (rows = n, act = dY) or dA^T (rows = k, act = X): sum over tokens of act^T . [hi + lo].
 int run_lora_grad(const Plan& P, const Split& sp, const uint16_t* act, int64_t m, int64_t rows, const uint16_t* hi,
                   const uint16_t* lo, int32_t r, float scale, float* out, int transpose, int accumulate, char* ws,
-                  cudaStream_t st) {
+                  cudaStream_t st, int grid_cap = 0) {
   GemmParams p = base_params(rows, P.r_pad, P.r_pad, cdiv(m, 64), sp);
   p.out = ws + P.off_part;
   p.ld_out = P.r_pad;
@@ -430,7 +431,7 @@ int run_lora_grad(const Plan& P, const Split& sp, const uint16_t* act, int64_t m
   ok = ok && tmap_2d(&maps.b, hi, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, 128);    // [m, r_pad], MN-major B
   ok = ok && tmap_2d(&maps.b2, lo, kBF16, P.r_pad, m, P.r_pad * 2, 64, 64, 128);
   if (!ok) return QLORA_ERR_CUDA;
-  cudaError_t e = launch_gemm(P.grad, p, maps, grid_of(p), st);
+  cudaError_t e = launch_gemm(P.grad, p, maps, grid_of(p, grid_cap), st);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   e = launch_grad_finalize(static_cast<const float*>(p.out), sp.splits, p.part_stride, rows, r, P.r_pad, scale, out,
                            transpose, accumulate, st);
@@ -508,6 +509,65 @@ int run_dx(const Plan& P, const DxLayer* L, int count, int64_t m, int64_t k, int
                            dx_dtype == QLORA_DTYPE_BF16, acc_dx ? 1 : 0, st) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
+}
+
+// SMs that a one-layer dX GEMM leaves idle and that can take the adapter gradients beside it
+// (0: run them after it). Only a dX GEMM with one split and no accumulation qualifies: it
+// writes dX directly and no fp32 partial. The gradients need enough SMs to end within the dX
+// GEMM's time: a low-rank K step streams 32 KB from memory, a weight K step runs a 256 x 512
+// x 64 MMA; the first is taken as about a third of the second.
+int dx_idle_sms(const Plan& P, int64_t m, int64_t n, int64_t k, bool acc_dx) {
+  constexpr int kMinIdle = 16;
+  if (acc_dx || P.bwd.splits != 1) return 0;
+  const int sms = num_sms();
+  const bool pair = wgemm_tile_rows(P.bn) == 256;
+  const int64_t units = cdiv(k, wgemm_tile_rows(P.bn)) * cdiv(m, P.bn);
+  const int64_t slots = pair ? wgemm_pair_slots() : sms;
+  const int64_t grid = (pair ? 2 : 1) * std::min<int64_t>(units, slots);
+  const int idle = static_cast<int>(sms - grid);
+  if (idle < kMinIdle) return 0;
+  const int64_t dx_steps = cdiv(units, slots) * (cdiv(n, 64) + P.r_pad / 64);
+  auto grad_steps = [&](const Split& sp, int64_t rows) {
+    return cdiv(cdiv(rows, 128) * sp.splits, idle) * (sp.kps + 1);
+  };
+  const int64_t side_steps = grad_steps(P.db, n) + grad_steps(P.da, k);
+  return (side_steps <= 3 * dx_steps) ? idle : 0;
+}
+
+// An internal stream (and a fork and a join event) per thread and CUDA context, on which a
+// backward runs work beside its dX GEMM. Created on the first call outside a stream capture;
+// a call under capture before that runs everything on the caller's stream.
+struct SideStream {
+  unsigned long long ctx = 0;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SideStream* side_stream(cudaStream_t st) {
+  thread_local std::vector<SideStream> cache;
+  const unsigned long long ctx = context_id();
+  if (ctx == 0) return nullptr;
+  for (SideStream& c : cache)
+    if (c.ctx == ctx) return &c;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return nullptr;
+  SideStream c;
+  c.ctx = ctx;
+  if (cudaStreamCreateWithFlags(&c.s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) != cudaSuccess) {
+    (void)cudaGetLastError();
+    if (c.join != nullptr) cudaEventDestroy(c.join);
+    if (c.fork != nullptr) cudaEventDestroy(c.fork);
+    if (c.s != nullptr) cudaStreamDestroy(c.s);
+    return nullptr;
+  }
+  cache.push_back(c);
+  return &cache.back();
 }
 
 // Workspace of a grouped backward: every layer's bf16(s G_l) (read together by the fused dX
@@ -766,20 +826,39 @@ int qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint
     if (rc != QLORA_OK) return rc;
   }
 
+  const float s_da = D.on ? s * D.keep : s;
+  const bool acc_dx = (flags & QLORA_BWD_ACCUMULATE_DX) != 0;
+  const int idle = (dX != nullptr && !D.on) ? dx_idle_sms(P, m, n, k, acc_dx) : 0;
+  SideStream* side = (idle > 0) ? side_stream(st) : nullptr;
+  if (side != nullptr) {
+    // dB and dA do not depend on dX: they run beside the dX GEMM on the SMs its grid leaves
+    // idle, with the same splits (the same partials, added in the same order). dX writes no
+    // fp32 partial here (one split, not accumulating), so the two share no workspace.
+    if (cudaEventRecord(side->fork, st) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    const DxLayer L{w, dY, A, sG};
+    int rc_dx = run_dx(P, &L, 1, m, k, r, true, dX, dx_dtype, false, wsb, st);
+    int rc_g = run_lora_grad(P, P.db, dY, m, n, u_hi, u_lo, r, s, dB, 0, acc_grads, wsb, side->s, idle);
+    if (rc_g == QLORA_OK) rc_g = run_lora_grad(P, P.da, Xl, m, k, g_hi, g_lo, r, s_da, dA, 1, acc_grads, wsb, side->s, idle);
+    // join even after a failed launch, so that the caller's stream (and a capture on it) ends
+    // after everything this call queued
+    if (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return (rc_dx != QLORA_OK) ? rc_dx : rc_g;
+  }
+
   if (dX != nullptr) {
     const DxLayer L{w, dY, A, sG};
-    rc = run_dx(P, &L, 1, m, k, r, !D.on, dX, dx_dtype, (flags & QLORA_BWD_ACCUMULATE_DX) != 0, wsb, st);
+    rc = run_dx(P, &L, 1, m, k, r, !D.on, dX, dx_dtype, acc_dx, wsb, st);
     if (rc != QLORA_OK) return rc;
     if (D.on) {
       rc = run_lora_up_masked(P, sG, m, k, A, r, D, dX, dx_dtype == QLORA_DTYPE_FP32, st);
       if (rc != QLORA_OK) return rc;
     }
   }
-
   rc = run_lora_grad(P, P.db, dY, m, n, u_hi, u_lo, r, s, dB, 0, acc_grads, wsb, st);
   if (rc != QLORA_OK) return rc;
-  rc = run_lora_grad(P, P.da, Xl, m, k, g_hi, g_lo, r, D.on ? s * D.keep : s, dA, 1, acc_grads, wsb, st);
-  return rc;
+  return run_lora_grad(P, P.da, Xl, m, k, g_hi, g_lo, r, s_da, dA, 1, acc_grads, wsb, st);
 }
 
 size_t qlora_linear_group_workspace_bytes(int32_t count, int64_t m, const int64_t* n, int64_t k, int32_t r) {

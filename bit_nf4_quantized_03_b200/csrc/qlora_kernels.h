@@ -45,6 +45,9 @@ Nf4Buckets nf4_buckets_from_midpoints(const float* mid);
 const Nf4Table& host_table();
 const Nf4Buckets& host_buckets();
 int host_num_sms();
+// Unique id of the calling thread's current CUDA context, 0 when none is current
+// (qlora_noalloc.cu; ids are never reused within a process).
+unsigned long long context_id();
 cudaError_t launch_dequantize(const uint8_t* codes, const ScaleSrc& ss, int64_t n_elem, const Nf4Table& tab,
                               uint16_t* out, int num_sms, cudaStream_t st);
 

@@ -61,6 +61,14 @@ unsigned long long current_context_id() {
   return id;
 }
 
+}  // namespace
+
+namespace qlora {
+unsigned long long context_id() { return current_context_id(); }
+}  // namespace qlora
+
+namespace {
+
 // Device address of the scratch array on the current device, looked up on the first
 // call per device and again whenever that device's context has changed since.
 int scratch_address(void** out) {

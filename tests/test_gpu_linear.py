@@ -3,6 +3,8 @@ the fp64 oracle on the same seeded inputs: relative Frobenius error <= 2e-3
 and max |error| <= 1e-2 x RMS of the reference, per output (Y, U, dX, dA, dB).
 fp32 outputs are checked at exactly those bounds; bf16 outputs with each
 element's bound widened by half a bf16 ulp of the reference."""
+import threading
+
 import numpy as np
 import pytest
 import torch
@@ -120,6 +122,70 @@ def test_repeat_calls_identical():
 def test_7b_q_proj_full():
     # 7B-shape q_proj: X 2048 x 4096 (batch 4 x seq 512), W 4096 x 4096, r = 64, alpha = 16
     _full_check(Layer(2048, 4096, 4096, 64))
+
+
+def test_backward_beside_dx_accumulating_grads():
+    # 512 tokens, W 256 x 2048: the CTA-pair dX GEMM (one split) takes 16 of 148 SMs, and dB and dA
+    # run beside it on the library's internal stream; accumulated into nonzero gradients
+    L = Layer(512, 256, 2048, 64)
+    Wd = L.oracle_weight()
+    _, U = L.fwd()
+    dX_ref, dA_ref, dB_ref = o.linear_backward(Wd, L.X, L.dY, L.A, L.B, L.alpha)
+    dX, dA1, dB1 = L.bwd(U)
+    check_close(dX.cpu(), dX_ref, "dX")
+    check_close(dA1.cpu(), dA_ref, "dA")
+    check_close(dB1.cpu(), dB_ref, "dB")
+    g = torch.Generator().manual_seed(5)
+    dA0 = torch.randn(L.r, L.k, generator=g) * 1e-2
+    dB0 = torch.randn(L.n, L.r, generator=g) * 1e-2
+    dA, dB = dA0.cuda(), dB0.cuda()
+    L.bwd(U, q.QLORA_DTYPE_FP32, q.QLORA_BWD_ACCUMULATE_GRADS, None, dA, dB)
+    check_close(dA.cpu(), dA_ref + dA0.double().numpy(), "dA+")
+    check_close(dB.cpu(), dB_ref + dB0.double().numpy(), "dB+")
+
+
+def _capture_bwd(L: Layer, U, outs):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=torch.cuda.Stream()):
+        q.qlora_linear_bwd(L.qw, L.Xd, L.dYd, L.Ad, L.Bd, L.r, L.alpha, U, outs[0], q.QLORA_DTYPE_FP32,
+                           outs[1], outs[2], 0, L.ws)
+    return g
+
+
+@pytest.mark.parametrize("shape", [(512, 256, 2048, 64), (2048, 4096, 4096, 64)])
+def test_backward_side_stream_same_bits_and_graph_replay(shape):
+    # With idle SMs beside the dX GEMM the backward forks dB and dA onto an internal stream and joins
+    # them back; a thread's first call under stream capture has no such stream yet and keeps all on
+    # the caller's stream. Eager, captured with the fork, and captured without it: the same bits.
+    L = Layer(*shape)
+    _, U = L.fwd()
+
+    def outs():
+        return tuple(torch.full(s, float("nan"), device="cuda") for s in ((L.m, L.k), (L.r, L.k), (L.n, L.r)))
+
+    eager = L.bwd(U)
+    forked = outs()
+    g_fork = _capture_bwd(L, U, forked)
+    single = outs()
+    box = {}
+
+    def in_thread():
+        try:
+            box["g"] = _capture_bwd(L, U, single)
+        except BaseException as e:      # reported by the assertion below
+            box["err"] = e
+
+    t = threading.Thread(target=in_thread)
+    t.start()
+    t.join()
+    assert "g" in box, box.get("err")
+    g_fork.replay()
+    box["g"].replay()
+    torch.cuda.synchronize()
+    q.qlora_check_device_error()
+    for name, a, b, c in zip(("dX", "dA", "dB"), eager, forked, single):
+        assert torch.equal(a, b), name + ": graph with the fork differs from the eager call"
+        assert torch.equal(a, c), name + ": one-stream graph differs from the eager call"
 
 
 def test_silu_gate_glue():
