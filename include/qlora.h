@@ -45,8 +45,10 @@
  * Conventions for every function:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never allocates device memory, never synchronizes, and keeps no state
- *    between calls other than a read-only level table and a device error word.
- *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *    between calls other than a read-only level table, a device error word and
+ *    the backward's internal stream and two events (per thread and context).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default), or
+ *    ordered with it through events (qlora_linear_bwd).
  *  - Argument errors are detected on the host before anything is enqueued
  *    and return QLORA_ERR_INVALID / QLORA_ERR_UNSUPPORTED / QLORA_ERR_WORKSPACE;
  *    a failed launch returns QLORA_ERR_CUDA.
@@ -221,6 +223,14 @@ int qlora_linear_fwd(const qlora_nf4_weight *w, const uint16_t *X, int64_t m, co
  * caller: the library holds no communicator). QLORA_BWD_ACCUMULATE_GRADS adds
  * into dA, dB instead, so several slices on one rank (gradient accumulation)
  * sum the same way before the exchange.
+ *
+ * Streams: when the dX GEMM leaves SMs idle (one split, dX not accumulated, no
+ * dropout), dA and dB are computed beside it on an internal stream of the
+ * library (one per host thread and CUDA context, created on that thread's first
+ * such call outside a stream capture). That stream waits on an event recorded
+ * on `stream`, and `stream` waits on one recorded after its work, so everything
+ * the call enqueues is ordered as if it ran on `stream` alone, under a CUDA
+ * graph capture too. The results are bit-identical either way.
  */
 int qlora_linear_bwd(const qlora_nf4_weight *w, const uint16_t *X, const uint16_t *dY, int64_t m,
                      const uint16_t *A, const uint16_t *B, int32_t r, float alpha, const float *U_saved,
