@@ -50,14 +50,20 @@ struct WCfg {
   static constexpr int kATile = 128 * 64 * 2;
   static constexpr int kBTile = TOK * 64 * 2;
   static constexpr int kRBytes = 4096;      // packed codes of one 128 x 64 weight tile
-  static constexpr int kThreads = (6 + 4 * (kGroups >= 2 ? kGroups : 2)) * 32;
+  // MMA-issuing threads: at 16 tokens the issue of the four small MMAs of every K step sets the
+  // pace, so a second warp issues every other K step into an accumulator of its own (the two
+  // are added in the epilogue); it is the warp after the dequantizers
+  static constexpr int kIssuers = (TOK == 16) ? 2 : 1;
+  static constexpr int kIssuer2Warp = 6 + 4 * (kGroups >= 2 ? kGroups : 2);
+  static constexpr int kThreads = (kIssuer2Warp + (kIssuers - 1)) * 32;
   static constexpr int kAccBufs = (2 * TOK <= 512) ? 2 : 1;   // double-buffer the accumulators when TMEM allows
-  static constexpr int kTmemCols = (kAccBufs * TOK <= 32) ? 32 : (kAccBufs * TOK <= 64) ? 64 : (kAccBufs * TOK <= 128) ? 128
-                                   : (kAccBufs * TOK <= 256) ? 256 : 512;
+  static constexpr int kAccCols = kAccBufs * kIssuers * TOK;
+  static constexpr int kTmemCols = (kAccCols <= 32) ? 32 : (kAccCols <= 64) ? 64 : (kAccCols <= 128) ? 128
+                                   : (kAccCols <= 256) ? 256 : 512;
   static constexpr int kSmemBytes = Stages * (kATile + kBTile + kRBytes) + 1024 + 256;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(BN % 32 == 0 || BN == 16, "epilogue reads 32 columns at a time");
-  static_assert(kAccBufs * TOK <= 512, "TMEM columns");
+  static_assert(kAccCols <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kGroups == 1 || (kGroups >= 2 && kStages % kGroups == 0), "the stage index modulo G picks the group");
 };
@@ -193,7 +199,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_full[a], C::kIssuers);      // one commit per issuing thread and unit
       mbar_init(&acc_empty[a], 4);
     }
     fence_mbar_init();
@@ -283,10 +289,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (C::kIssuers == 2 && warp == C::kIssuer2Warp)) {
+    // ------------------------------------------------------------ MMA issuer(s)
+    // issuer e takes the unit's K steps i with i % kIssuers == e, into its own accumulator
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(C::BN, C::Bwd, false);
+      const int e = (warp == 1) ? 0 : 1;
       int stage = 0;
       uint32_t ph = 0;
       int acc = 0;
@@ -297,8 +305,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         wdecode(p, u, mb, nb, split, kt0, nmain, next);
         if (!mbar_wait(&acc_empty[acc], aph ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::TOK);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((acc * C::kIssuers + e) * C::TOK);
         for (int i = 0; i < nmain + next; ++i) {
+          if (i % C::kIssuers != e) {
+            if (++stage == C::Stages) { stage = 0; ph ^= 1; }
+            continue;
+          }
           if (!mbar_wait(&tma_full[stage], ph)) { ok = false; break; }
           if (!mbar_wait(&deq_full[stage], ph)) { ok = false; break; }
           // operands reach the MMA through the barriers alone (TMA completion; the
@@ -312,7 +324,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 #pragma unroll
             for (int t = 0; t < C::NAcc; ++t) {
               const uint64_t bd = umma_desc_sw128(b_addr + t * (C::BN * 128) + kk * 32, 16, 1024);
-              umma_bf16(d_tmem + t * C::BN, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+              umma_bf16(d_tmem + t * C::BN, ad, bd, idesc, (i > e || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(&empty[stage]);
@@ -335,11 +347,21 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (!mbar_wait(&acc_full[acc], aph)) break;
       tc_fence_after();
       const int feat = mb * 128 + q * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::TOK);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * C::kIssuers * C::TOK);
       if (C::BN == 16) {
         uint32_t v[32];
         tmem_ld_32x32b_x16(t_row, v);
-        tmem_ld_wait();
+        if (C::kIssuers == 2 && nmain + next > 1) {
+          // the second issuer's accumulator (written only when the unit has a second K step)
+          uint32_t w[32];
+          tmem_ld_32x32b_x16(t_row + C::TOK, w);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__fadd_rn(__uint_as_float(v[j]), __uint_as_float(w[j])));
+        } else {
+          tmem_ld_wait();
+        }
         wstore<16>(p, split, feat, nb * C::TOK, v);
       } else {
 #pragma unroll 1
