@@ -26,6 +26,8 @@
 //   warps 6-    dequantizers: groups of four warps take turns on the K steps
 //               (three groups in the single-CTA kernel, two in the pair);
 //               one thread expands one row's 64-block per step
+//   last warp   (single-CTA kernel at 16 tokens) a second tcgen05.mma issuer:
+//               every other K step, into an accumulator of its own
 #include <cudaTypedefs.h>
 
 #include <cstring>
